@@ -1,0 +1,225 @@
+/*
+ * tfpaged.h - C ABI of a B200 (sm_100a) library for multi-stream attention
+ * over a paged bf16 KV cache.
+ *
+ * Sources of the operations (TensorFold pull requests, by title and section):
+ *  - #1503 "lfm2_moe CUDA: attention pages from the shared KV pool, and the
+ *    prompt cache", commit list: one launch a layer over every stream's rows
+ *    from a table of cache addresses, row offsets and key counts (the
+ *    segment table); split-KV chunk and merge bodies over paged caches
+ *    (tf_paged_attn_chunk_segs_*, tf_paged_attn_merge_segs_*); lfm2_argmax
+ *    (first largest logit, ties to the lower id, nonfinite rows flagged);
+ *    forward refuses rows past a slot's pages.
+ *  - #1653 "spark25 CUDA: the full layers' caches in pages of the core pool",
+ *    PR body: decode reads K/V through the whole page table, prompt rows
+ *    through the slot's row (tf_wrows_prompt_256_p32_pg); pages of 32 and 256
+ *    positions; review thread: the paged merge's nonfinite-head handling and
+ *    the per-chunk page lookup hoisted out of the key loop.
+ *  - #1562 "Qwen3.6 MTP drafter on CUDA: draft a shared round's streams
+ *    together", PR body: many streams' rows in one launch, each over its own
+ *    ring of slots (tf_q36m_attn_rows); slots stepped with a wrap, the next
+ *    group of slots in flight while the current one folds.
+ *
+ * Conventions shared by every call:
+ *  - All pointers except those named *_host are DEVICE pointers.  The caller
+ *    owns every buffer; the library allocates nothing, keeps no mutable
+ *    global state and never synchronizes: work is enqueued on `stream`
+ *    (NULL = the legacy default stream) and the call returns.
+ *  - bf16 data is passed as raw 16-bit patterns (`const void*`).
+ *  - The return value reports host-checkable errors only (bad sizes, null
+ *    pointers, unsupported shapes, misaligned buffers and, when a host copy
+ *    of a table is given, table errors).  Nothing is launched when it is not
+ *    TF_OK.
+ *  - Errors the device finds in a table (bad segment, keys past a stream's
+ *    pages, a page id outside the pool, too many splits) are OR-ed as
+ *    TF_DEV_* bits into the caller's uint32 `status` word (device memory;
+ *    the caller zeroes it); the affected work is skipped and, where it has
+ *    outputs, flagged.  No kernel ever traps, asserts or spins unbounded.
+ *  - Nonfinite data is not an error: the affected (row, head) is reported in
+ *    the flags output and its output holds NaN.
+ *
+ * Data layout (a reading: the pages give no layout):
+ *  - q:      bf16 [n_rows_total][Hq][D]
+ *  - K pool: bf16 [n_pages][Hkv][page_size][D], V pool alike, separate arrays
+ *  - page table: int32; stream s owns entries [pt_base, pt_base + n_pages)
+ *  - q-head h reads kv-head h / (Hq / Hkv)
+ *  - row i of a stream with n_rows new rows and n_keys keys sees keys
+ *    [0, n_keys - n_rows + i + 1) (causal within the new rows)
+ *  - partials: o f32 [n_rows_total][Hq][n_splits_max][D] (unnormalised
+ *    sum e^(s - m) v), m f32 and l f32 [n_rows_total][Hq][n_splits_max]
+ *    (m = max score in natural-log units, l = sum e^(s - m)), flag u8 alike.
+ */
+#ifndef TFPAGED_H
+#define TFPAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TF_API __attribute__((visibility("default")))
+#else
+#define TF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream (cudaStream_t / CUstream). */
+typedef struct CUstream_st *tf_stream_t;
+
+typedef enum {
+    TF_OK = 0,
+    TF_ERR_ARG = 1,         /* a null pointer, a negative or inconsistent size */
+    TF_ERR_PAST_PAGES = 2,  /* a host table asks for keys past a stream's pages */
+    TF_ERR_BAD_PAGE = 3,    /* a host table names a page outside the pool */
+    TF_ERR_UNSUPPORTED = 4, /* head dim, page size or head counts outside what is built */
+    TF_ERR_CUDA = 5,        /* a launch failed (cudaGetLastError after the launch) */
+    TF_ERR_ALIGN = 6,       /* a buffer is not aligned as documented */
+    TF_ERR_WORKSPACE = 7    /* the workspace is smaller than the size query returns */
+} tf_status;
+
+/* Bits OR-ed into the device status word. */
+#define TF_DEV_BAD_SEG 0x1u    /* a segment's rows or page range fall outside the buffers */
+#define TF_DEV_PAST_PAGES 0x2u /* n_keys > n_pages * page_size (the pages' PastPages refusal) */
+#define TF_DEV_BAD_PAGE 0x4u   /* a page id outside [0, n_pages of the pool) */
+#define TF_DEV_SPLITS 0x8u     /* a stream needs more partials than n_splits_max */
+
+/* One stream's entry in the segment table (device array, int32 fields). */
+typedef struct {
+    int32_t q_row;   /* first row of the stream in q / partials / out */
+    int32_t n_rows;  /* its query rows this call (0 = nothing to do) */
+    int32_t n_keys;  /* keys visible to its last row, its new rows included */
+    int32_t pt_base; /* first entry of its pages in the page table */
+    int32_t n_pages; /* how many page-table entries it owns */
+} tf_seg;
+
+/* One row's entry in a ring table (device array).  Slots [base, base+size)
+ * of the ring arrays form the ring; `head` is the slot the next key will be
+ * written to, and the row attends to the n_valid slots written just before
+ * it, oldest first: slot_j = (head - n_valid + j) mod size. */
+typedef struct {
+    int64_t base;
+    int32_t q_row;
+    int32_t size;
+    int32_t head;
+    int32_t n_valid;
+} tf_ring_seg;
+
+enum { TF_OUT_F32 = 0, TF_OUT_BF16 = 1 };
+
+/*
+ * Split-KV partials of paged attention for every row of every stream in one
+ * launch (the segment kernels of #1503, commit list; decode and verify reads
+ * through the whole page table, #1653 PR body).
+ *
+ * Partial c of stream s covers keys [c*K, min((c+1)*K, n_keys)) where K =
+ * split_keys when split_keys > 0, else K = ceil(ceil(n_keys/n_splits_max)/P)*P.
+ * For each row i and q-head h it writes m, l, o over the keys of that range
+ * that the row sees, and flag = a visible score, or a visible value row, or
+ * o is nonfinite.  A partial holding no visible key has m = -inf, l = 0 and
+ * o = 0; a slot c at or past the stream's partial count gets m = -inf, l = 0,
+ * flag = 0 and its o is left unwritten.
+ *
+ *  q          bf16 [n_rows_total][n_q_heads][head_dim]
+ *  k_pool, v_pool  bf16 [n_pages][n_kv_heads][page_size][head_dim], 16-byte aligned
+ *  page_table int32 [page_table_len]
+ *  segs       tf_seg [n_segs] (device);  segs_host: optional host copy of
+ *             the same table; when given it is validated first (and page ids
+ *             too, when page_table_host is given)
+ *  scale      score scale (1/sqrt(head_dim) for plain attention)
+ *  part_*     outputs as laid out above
+ *  status     uint32 device word for TF_DEV_* bits (not cleared by the call)
+ *
+ * Supported: head_dim in {64, 128, 256}; page_size a power of two in
+ * [8, 1024]; n_q_heads a multiple of n_kv_heads; q, pools 16-byte aligned.
+ */
+TF_API tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                               const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                               int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                               const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                               const int32_t *page_table_host, float scale, int32_t split_keys,
+                               int32_t n_splits_max, float *part_o, float *part_m, float *part_l,
+                               uint8_t *part_flag, uint32_t *status, tf_stream_t stream);
+
+/*
+ * Fold partials into the final output (the merge bodies of #1503, commit
+ * list; the nonfinite-head handling of #1653, review thread).  Per (row, head):
+ * M = max m_c over partials with l_c > 0, L = sum e^(m_c - M) l_c,
+ * out = sum e^(m_c - M) o_c / L; flag = OR of the partials' flags, or out
+ * nonfinite, or no partial holds a key; a flagged head's out is NaN.
+ * o_c is read only for partials with l_c > 0.
+ *
+ *  out   f32 [n_rows_total][n_q_heads][head_dim];  flags u8 [n_rows_total][n_q_heads]
+ */
+TF_API tf_status tf_attn_merge(const float *part_o, const float *part_m, const float *part_l, const uint8_t *part_flag,
+                        int32_t n_rows_total, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max, float *out,
+                        uint8_t *flags, tf_stream_t stream);
+
+/*
+ * Causal prompt chunk through one stream's page-table row (the _pg prompt
+ * kernel of #1653, commit list and PR body): rows i = 0..n_rows-1 of the
+ * chunk (q/out rows seg.q_row + i) attend to keys [0, n_keys - n_rows + i + 1),
+ * every key already in the pool.  Scores and sums in fp32 on the tensor
+ * cores; out is bf16 (out_dtype TF_OUT_BF16) or f32 [rows][Hq][D].
+ * flags (nullable) u8 [rows][Hq] as for the merge; a flagged head's out is NaN.
+ *
+ *  seg_host  the stream's segment, in HOST memory (the chunk's size sets the grid)
+ *
+ * Supported: head_dim in {64, 128, 256}; page sizes as for decode.
+ */
+TF_API tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                               const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                               int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                               const tf_seg *seg_host, float scale, void *out, int32_t out_dtype, uint8_t *flags,
+                               uint32_t *status, tf_stream_t stream);
+
+/*
+ * Attention of many rows, each over its own ring of slots, in one launch
+ * (tf_q36m_attn_rows of #1562, PR body), split over the ring's valid slots
+ * into partials of split_slots slots and merged into out.
+ *
+ *  q          bf16 [n_rows_total][n_q_heads][head_dim]
+ *  ring_k, ring_v  bf16 [ring_slots_total][n_kv_heads][head_dim], 16-byte aligned
+ *  rsegs      tf_ring_seg [n_segs] (device); rsegs_host: optional host copy, validated
+ *  workspace  device scratch of at least tf_ring_workspace_bytes(...) bytes;
+ *             it holds the partials between the partial and merge kernels,
+ *             laid out per table entry, and needs no initialisation
+ *  out        f32 [n_rows_total][n_q_heads][head_dim];  flags u8 [n_rows_total][n_q_heads]
+ *             Only the rows the table names are written.
+ *
+ * Supported: head_dim in {64, 128, 256}; n_q_heads a multiple of n_kv_heads;
+ * split_slots >= 16; n_splits_max >= ceil(n_valid / split_slots) for every
+ * entry (else TF_DEV_SPLITS and the entry is skipped).
+ */
+TF_API tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *ring_k, const void *ring_v,
+                       int64_t ring_slots_total, int32_t n_kv_heads, int32_t head_dim, const tf_ring_seg *rsegs,
+                       int32_t n_segs, const tf_ring_seg *rsegs_host, float scale, int32_t split_slots,
+                       int32_t n_splits_max, void *workspace, size_t workspace_bytes, float *out, uint8_t *flags,
+                       uint32_t *status, tf_stream_t stream);
+
+/* Workspace bytes tf_ring_attn needs for these sizes (0 on bad sizes). */
+TF_API size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max);
+
+/*
+ * Greedy row argmax (lfm2_argmax of #1503, commit list): for each of n_rows
+ * rows of n_cols bf16 logits (row stride ld elements), ids[r] = the lowest
+ * column holding the row's largest value, values compared as real numbers
+ * (-0 equals +0); flags[r] = 1 and ids[r] = -1 when the row holds a NaN or
+ * an infinity.  One launch; each row is split over a cluster of CTAs that
+ * reduce through distributed shared memory, so no workspace is needed.
+ */
+TF_API tf_status tf_argmax_rows(const void *logits, int32_t n_rows, int32_t n_cols, int64_t ld, int32_t *ids,
+                         uint8_t *flags, tf_stream_t stream);
+
+/* Text of a status code (static storage). */
+TF_API const char *tf_status_str(tf_status s);
+
+/* ABI version of this header: bumped when a signature changes. */
+TF_API int32_t tf_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TFPAGED_H */

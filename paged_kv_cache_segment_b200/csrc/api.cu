@@ -1,0 +1,306 @@
+// api.cu - the extern "C" entry points declared in include/tfpaged.h: argument
+// checks on the host, then stream-ordered kernel launches.  Nothing here
+// allocates, synchronizes or keeps state between calls.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tf_internal.h"
+
+using namespace tfp;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int log2_exact(int x) {
+    if (x <= 0 || (x & (x - 1))) return -1;
+    int r = 0;
+    while ((1 << r) < x) ++r;
+    return r;
+}
+
+bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
+
+tf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TF_OK : TF_ERR_CUDA; }
+
+int split_len(int n_keys, int split_keys, int n_splits_max, int page_size) {
+    if (split_keys > 0) return split_keys;
+    int per = (n_keys + n_splits_max - 1) / n_splits_max;
+    return (per + page_size - 1) / page_size * page_size;
+}
+
+// Checks of a host copy of a segment table; see tf_paged_attn_decode.
+tf_status check_segs_host(const tf_seg *sh, int n_segs, int n_rows_total, int page_table_len, int page_size,
+                          int n_pages, const int32_t *pt_host, int split_keys, int n_splits_max, int *max_rows) {
+    int mr = 0;
+    for (int s = 0; s < n_segs; ++s) {
+        const tf_seg e = sh[s];
+        if (e.q_row < 0 || e.n_rows < 0 || (int64_t)e.q_row + e.n_rows > n_rows_total || e.n_keys < e.n_rows ||
+            e.pt_base < 0 || e.n_pages < 0 || (int64_t)e.pt_base + e.n_pages > page_table_len)
+            return TF_ERR_ARG;
+        if ((int64_t)e.n_keys > (int64_t)e.n_pages * page_size) return TF_ERR_PAST_PAGES;
+        if (e.n_rows > 0 && n_splits_max > 0) {
+            const int per = split_len(e.n_keys, split_keys, n_splits_max, page_size);
+            if ((e.n_keys + per - 1) / per > n_splits_max) return TF_ERR_ARG;
+        }
+        if (pt_host) {
+            const int used = (e.n_keys + page_size - 1) / page_size;
+            for (int k = 0; k < used; ++k) {
+                const int pid = pt_host[e.pt_base + k];
+                if (pid < 0 || pid >= n_pages) return TF_ERR_BAD_PAGE;
+            }
+        }
+        if (e.n_rows > mr) mr = e.n_rows;
+    }
+    *max_rows = mr;
+    return TF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                               const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                               int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                               const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                               const int32_t *page_table_host, float scale, int32_t split_keys,
+                               int32_t n_splits_max, float *part_o, float *part_m, float *part_l,
+                               uint8_t *part_flag, uint32_t *status, tf_stream_t stream) {
+    if (n_rows_total < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_pages < 0 || page_table_len < 0 || n_segs < 0 ||
+        split_keys < 0 || n_splits_max <= 0 || !std::isfinite(scale))
+        return TF_ERR_ARG;
+    if (n_q_heads % n_kv_heads != 0) return TF_ERR_UNSUPPORTED;
+    if (!head_dim_ok(head_dim)) return TF_ERR_UNSUPPORTED;
+    const int lp = log2_exact(page_size);
+    if (lp < 3 || lp > 10) return TF_ERR_UNSUPPORTED;
+    if (split_keys > 0 && split_keys < 16) return TF_ERR_UNSUPPORTED;
+    if (n_segs > 65535) return TF_ERR_UNSUPPORTED;
+    if (n_segs == 0 || n_rows_total == 0) return TF_OK;
+    if (!q || !k_pool || !v_pool || !page_table || !segs || !part_o || !part_m || !part_l || !part_flag || !status)
+        return TF_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(part_o)) return TF_ERR_ALIGN;
+    const int group = n_q_heads / n_kv_heads;
+    int max_rows = n_rows_total;
+    if (segs_host) {
+        const tf_status st = check_segs_host(segs_host, n_segs, n_rows_total, page_table_len, page_size, n_pages,
+                                             page_table_host, split_keys, n_splits_max, &max_rows);
+        if (st != TF_OK) return st;
+        if (max_rows == 0) return TF_OK;
+    }
+    const int64_t n_qgroups = ((int64_t)max_rows * group + 63) / 64;
+    if (n_qgroups * n_kv_heads > 65535 || n_splits_max > (1 << 30)) return TF_ERR_UNSUPPORTED;
+
+    AttnParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.n_rows_total = n_rows_total;
+    p.hq = n_q_heads;
+    p.hkv = n_kv_heads;
+    p.group = group;
+    p.k = static_cast<const uint16_t *>(k_pool);
+    p.v = static_cast<const uint16_t *>(v_pool);
+    p.n_pages = n_pages;
+    p.log2_page = lp;
+    p.pt_len = page_table_len;
+    p.page_table = page_table;
+    p.segs = segs;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.split_keys = split_keys;
+    p.n_splits_max = n_splits_max;
+    p.n_qgroups = (int)n_qgroups;
+    p.part_o = part_o;
+    p.part_m = part_m;
+    p.part_l = part_l;
+    p.part_flag = part_flag;
+    p.status = status;
+    const dim3 grid((unsigned)n_splits_max, (unsigned)(n_qgroups * n_kv_heads), (unsigned)n_segs);
+    return cuda_status(launch_attn_partial(p, head_dim, false, false, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tf_status tf_attn_merge(const float *part_o, const float *part_m, const float *part_l, const uint8_t *part_flag,
+                        int32_t n_rows_total, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max, float *out,
+                        uint8_t *flags, tf_stream_t stream) {
+    if (n_rows_total < 0 || n_q_heads <= 0 || n_splits_max <= 0) return TF_ERR_ARG;
+    if (!head_dim_ok(head_dim)) return TF_ERR_UNSUPPORTED;
+    if (n_rows_total == 0) return TF_OK;
+    if (!part_o || !part_m || !part_l || !part_flag || !out || !flags) return TF_ERR_ARG;
+    if (!aligned16(part_o) || !aligned16(out)) return TF_ERR_ALIGN;
+    MergeParams p{};
+    p.part_o = part_o;
+    p.part_m = part_m;
+    p.part_l = part_l;
+    p.part_flag = part_flag;
+    p.n_units = (int64_t)n_rows_total * n_q_heads;
+    p.n_parts = n_splits_max;
+    p.hq = n_q_heads;
+    p.n_rows_total = n_rows_total;
+    p.out = out;
+    p.flags = flags;
+    return cuda_status(launch_merge(p, head_dim, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                               const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                               int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                               const tf_seg *seg_host, float scale, void *out, int32_t out_dtype, uint8_t *flags,
+                               uint32_t *status, tf_stream_t stream) {
+    if (!seg_host || n_rows_total < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_pages < 0 || page_table_len < 0 ||
+        !std::isfinite(scale))
+        return TF_ERR_ARG;
+    if (out_dtype != TF_OUT_F32 && out_dtype != TF_OUT_BF16) return TF_ERR_ARG;
+    if (n_q_heads % n_kv_heads != 0 || !head_dim_ok(head_dim)) return TF_ERR_UNSUPPORTED;
+    const int lp = log2_exact(page_size);
+    if (lp < 3 || lp > 10) return TF_ERR_UNSUPPORTED;
+    int max_rows = 0;
+    const tf_status st =
+        check_segs_host(seg_host, 1, n_rows_total, page_table_len, page_size, n_pages, nullptr, 0, 1, &max_rows);
+    if (st != TF_OK) return st;
+    if (max_rows == 0) return TF_OK;
+    if (!q || !k_pool || !v_pool || !page_table || !out || !status) return TF_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(out)) return TF_ERR_ALIGN;
+    const int group = n_q_heads / n_kv_heads;
+    const int64_t n_qgroups = ((int64_t)max_rows * group + 63) / 64;
+    if (n_qgroups * n_kv_heads > 65535) return TF_ERR_UNSUPPORTED;
+
+    AttnParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.n_rows_total = n_rows_total;
+    p.hq = n_q_heads;
+    p.hkv = n_kv_heads;
+    p.group = group;
+    p.k = static_cast<const uint16_t *>(k_pool);
+    p.v = static_cast<const uint16_t *>(v_pool);
+    p.n_pages = n_pages;
+    p.log2_page = lp;
+    p.pt_len = page_table_len;
+    p.page_table = page_table;
+    p.seg0 = *seg_host;
+    p.seg_inline = 1;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.split_keys = 0;
+    p.n_splits_max = 1;
+    p.n_qgroups = (int)n_qgroups;
+    p.out = out;
+    p.out_bf16 = out_dtype == TF_OUT_BF16;
+    p.out_flags = flags;
+    p.status = status;
+    const dim3 grid(1u, (unsigned)(n_qgroups * n_kv_heads), 1u);
+    return cuda_status(launch_attn_partial(p, head_dim, false, true, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max) {
+    if (n_segs < 0 || n_q_heads <= 0 || head_dim <= 0 || n_splits_max <= 0) return 0;
+    const size_t parts = (size_t)n_segs * n_q_heads * n_splits_max;
+    const size_t o = parts * head_dim * sizeof(float);
+    const size_t ml = 2 * parts * sizeof(float);
+    return ((o + ml + parts + 255) / 256) * 256;
+}
+
+tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *ring_k, const void *ring_v,
+                       int64_t ring_slots_total, int32_t n_kv_heads, int32_t head_dim, const tf_ring_seg *rsegs,
+                       int32_t n_segs, const tf_ring_seg *rsegs_host, float scale, int32_t split_slots,
+                       int32_t n_splits_max, void *workspace, size_t workspace_bytes, float *out, uint8_t *flags,
+                       uint32_t *status, tf_stream_t stream) {
+    if (n_rows_total < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || ring_slots_total < 0 || n_segs < 0 ||
+        n_splits_max <= 0 || !std::isfinite(scale))
+        return TF_ERR_ARG;
+    if (n_q_heads % n_kv_heads != 0 || !head_dim_ok(head_dim) || split_slots < 16) return TF_ERR_UNSUPPORTED;
+    if (n_segs > 65535) return TF_ERR_UNSUPPORTED;
+    if (n_segs == 0) return TF_OK;
+    if (!q || !ring_k || !ring_v || !rsegs || !workspace || !out || !flags || !status) return TF_ERR_ARG;
+    if (!aligned16(q) || !aligned16(ring_k) || !aligned16(ring_v) || !aligned16(out) || !aligned16(workspace))
+        return TF_ERR_ALIGN;
+    if (workspace_bytes < tf_ring_workspace_bytes(n_segs, n_q_heads, head_dim, n_splits_max)) return TF_ERR_WORKSPACE;
+    if (rsegs_host) {
+        for (int s = 0; s < n_segs; ++s) {
+            const tf_ring_seg e = rsegs_host[s];
+            if (e.q_row < 0 || e.q_row >= n_rows_total || e.size <= 0 || e.n_valid < 1 || e.n_valid > e.size ||
+                e.head < 0 || e.head >= e.size || e.base < 0 || e.base + e.size > ring_slots_total)
+                return TF_ERR_ARG;
+            if ((e.n_valid + split_slots - 1) / split_slots > n_splits_max) return TF_ERR_ARG;
+        }
+    }
+    const int group = n_q_heads / n_kv_heads;
+    const int n_qgroups = (group + 63) / 64;
+    if ((int64_t)n_qgroups * n_kv_heads > 65535) return TF_ERR_UNSUPPORTED;
+    const size_t parts = (size_t)n_segs * n_q_heads * n_splits_max;
+    float *po = static_cast<float *>(workspace);
+    float *pm = po + parts * head_dim;
+    float *pl = pm + parts;
+    uint8_t *pf = reinterpret_cast<uint8_t *>(pl + parts);
+
+    AttnParams p{};
+    p.q = static_cast<const uint16_t *>(q);
+    p.n_rows_total = n_rows_total;
+    p.hq = n_q_heads;
+    p.hkv = n_kv_heads;
+    p.group = group;
+    p.k = static_cast<const uint16_t *>(ring_k);
+    p.v = static_cast<const uint16_t *>(ring_v);
+    p.rsegs = rsegs;
+    p.ring_slots_total = ring_slots_total;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.split_keys = split_slots;
+    p.n_splits_max = n_splits_max;
+    p.n_qgroups = n_qgroups;
+    p.part_o = po;
+    p.part_m = pm;
+    p.part_l = pl;
+    p.part_flag = pf;
+    p.status = status;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((unsigned)n_splits_max, (unsigned)(n_qgroups * n_kv_heads), (unsigned)n_segs);
+    cudaError_t e = launch_attn_partial(p, head_dim, true, false, grid, st);
+    if (e != cudaSuccess) return TF_ERR_CUDA;
+    MergeParams mp{};
+    mp.part_o = po;
+    mp.part_m = pm;
+    mp.part_l = pl;
+    mp.part_flag = pf;
+    mp.n_units = (int64_t)n_segs * n_q_heads;
+    mp.n_parts = n_splits_max;
+    mp.hq = n_q_heads;
+    mp.n_rows_total = n_rows_total;
+    mp.rsegs = rsegs;
+    mp.split_slots = split_slots;
+    mp.ring_slots_total = ring_slots_total;
+    mp.out = out;
+    mp.flags = flags;
+    return cuda_status(launch_merge(mp, head_dim, true, st));
+}
+
+tf_status tf_argmax_rows(const void *logits, int32_t n_rows, int32_t n_cols, int64_t ld, int32_t *ids,
+                         uint8_t *flags, tf_stream_t stream) {
+    if (n_rows < 0 || n_cols <= 0 || ld < n_cols) return TF_ERR_ARG;
+    if (n_rows == 0) return TF_OK;
+    if (!logits || !ids || !flags) return TF_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(logits) & 1u) != 0) return TF_ERR_ALIGN;
+    ArgmaxParams p{};
+    p.logits = static_cast<const uint16_t *>(logits);
+    p.n_rows = n_rows;
+    p.n_cols = n_cols;
+    p.ld = ld;
+    p.ids = ids;
+    p.flags = flags;
+    const bool vec = aligned16(logits) && (ld % 8) == 0;
+    return cuda_status(launch_argmax(p, vec, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char *tf_status_str(tf_status s) {
+    switch (s) {
+        case TF_OK: return "ok";
+        case TF_ERR_ARG: return "bad argument";
+        case TF_ERR_PAST_PAGES: return "keys past a stream's pages";
+        case TF_ERR_BAD_PAGE: return "page id outside the pool";
+        case TF_ERR_UNSUPPORTED: return "unsupported shape";
+        case TF_ERR_CUDA: return "CUDA launch error";
+        case TF_ERR_ALIGN: return "misaligned buffer";
+        case TF_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+int32_t tf_abi_version(void) { return 1; }
+
+}  // extern "C"

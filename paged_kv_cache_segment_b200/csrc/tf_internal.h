@@ -1,0 +1,65 @@
+// tf_internal.h - parameter blocks and launchers shared between the C-ABI
+// entry points (api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/tfpaged.h"
+
+namespace tfp {
+
+// Parameters of the split-KV attention kernel (paged or ring source).
+struct AttnParams {
+    const uint16_t *q;
+    int n_rows_total, hq, hkv, group;
+    const uint16_t *k, *v;  // pool [pages][Hkv][P][D] or ring [slots][Hkv][D]
+    // paged source
+    int n_pages, log2_page, pt_len;
+    const int32_t *page_table;
+    const tf_seg *segs;
+    tf_seg seg0;     // used instead of segs[0] when seg_inline != 0 (one-stream prompt calls)
+    int seg_inline;
+    // ring source
+    const tf_ring_seg *rsegs;
+    int64_t ring_slots_total;
+    float scale_log2;  // scale * log2(e)
+    int split_keys, n_splits_max, n_qgroups;
+    // partial outputs [unit][n_splits_max](*D)
+    float *part_o, *part_m, *part_l;
+    uint8_t *part_flag;
+    // direct outputs [row][Hq](*D)
+    void *out;
+    int out_bf16;
+    uint8_t *out_flags;
+    uint32_t *status;
+};
+
+struct MergeParams {
+    const float *part_o, *part_m, *part_l;
+    const uint8_t *part_flag;
+    int64_t n_units;  // units of partials (rows x heads, or ring entries x heads)
+    int n_parts, hq, n_rows_total;
+    const tf_ring_seg *rsegs;  // ring merge: unit s * Hq + h writes row rsegs[s].q_row
+    int split_slots;           // ring merge: partials of entry s are ceil(n_valid / split_slots)
+    int64_t ring_slots_total;
+    float *out;
+    uint8_t *flags;
+};
+
+struct ArgmaxParams {
+    const uint16_t *logits;
+    int n_rows, n_cols;
+    int64_t ld;
+    int32_t *ids;
+    uint8_t *flags;
+};
+
+cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bool direct, dim3 grid,
+                                cudaStream_t st);
+cudaError_t launch_merge(const MergeParams &p, int head_dim, bool ring, cudaStream_t st);
+cudaError_t launch_argmax(const ArgmaxParams &p, bool vec, cudaStream_t st);
+
+constexpr int kArgmaxCluster = 8;
+
+}  // namespace tfp

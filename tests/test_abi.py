@@ -1,0 +1,90 @@
+"""The C-ABI library loads and exports every symbol include/tfpaged.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import paged_kv_cache_segment_b200 as tf
+from paged_kv_cache_segment_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"TF_API\s+[\w\s\*]+?\b(tf_\w+)\s*\(", src)
+    return names
+
+
+def test_header_declares_the_calls():
+    names = declared_symbols()
+    for n in ("tf_paged_attn_decode", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn", "tf_argmax_rows"):
+        assert n in names
+    assert set(binding.EXPORTS) == set(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tf.load()
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+    assert tf.tf_abi_version() == 1
+    assert tf.tf_status_str(0) == "ok"
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case below fails a host check first
+
+
+def call_decode(**kw):
+    lib = tf.load()
+    a = dict(q=FAKE, rows=4, hq=8, k=FAKE, v=FAKE, n_pages=16, psz=16, hkv=2, d=64, pt=FAKE, pt_len=8, segs=FAKE,
+             n_segs=2, segs_host=None, pt_host=None, scale=0.125, split=0, nsm=2, po=FAKE, pm=FAKE, pl=FAKE, pf=FAKE,
+             st=FAKE, stream=None)
+    a.update(kw)
+    return lib.tf_paged_attn_decode(*a.values())
+
+
+def test_host_checks_of_decode():
+    assert call_decode(d=96) == 4  # unsupported head dim
+    assert call_decode(psz=24) == 4  # page size not a power of two
+    assert call_decode(hq=7) == 4  # Hq not a multiple of Hkv
+    assert call_decode(nsm=0) == 1
+    assert call_decode(q=ctypes.c_void_p(0x10008)) == 6  # misaligned
+    assert call_decode(scale=float("nan")) == 1
+    assert call_decode(n_segs=0) == 0  # nothing to do, nothing launched
+    segs = np.array([[0, 1, 37, 0, 3], [1, 1, 70, 3, 5]], np.int32)
+    assert call_decode(segs_host=segs.ctypes.data_as(ctypes.c_void_p), n_segs=2, pt_len=8,
+                       nsm=1, split=16) == 1  # needs more than one partial
+    bad = segs.copy()
+    bad[0, 2] = 49  # 3 pages of 16 hold 48 keys
+    assert call_decode(segs_host=bad.ctypes.data_as(ctypes.c_void_p)) == 2
+    pt = np.arange(8, dtype=np.int32)
+    pt[4] = 16
+    assert call_decode(segs_host=segs.ctypes.data_as(ctypes.c_void_p), pt_host=pt.ctypes.data_as(ctypes.c_void_p)) == 3
+    zero_rows = segs.copy()
+    zero_rows[:, 1] = 0
+    assert call_decode(segs_host=zero_rows.ctypes.data_as(ctypes.c_void_p)) == 0
+
+
+def test_host_checks_of_other_calls():
+    lib = tf.load()
+    assert lib.tf_attn_merge(FAKE, FAKE, FAKE, FAKE, 4, 8, 100, 2, FAKE, FAKE, None) == 4
+    assert lib.tf_argmax_rows(FAKE, 4, 0, 10, FAKE, FAKE, None) == 1
+    assert lib.tf_argmax_rows(FAKE, 4, 20, 10, FAKE, FAKE, None) == 1
+    assert lib.tf_argmax_rows(FAKE, 0, 20, 20, FAKE, FAKE, None) == 0
+    assert lib.tf_ring_workspace_bytes(17, 16, 256, 17) >= 17 * 16 * 17 * (256 + 2) * 4
+    rs = np.zeros(1, binding.RING_SEG_DTYPE)
+    rs[0] = (0, 0, 100, 5, 101)  # more valid slots than the ring holds
+    ws = lib.tf_ring_workspace_bytes(1, 8, 64, 4)
+    assert lib.tf_ring_attn(FAKE, 1, 8, FAKE, FAKE, 100, 2, 64, FAKE, 1, rs.ctypes.data_as(ctypes.c_void_p), 0.1, 64,
+                            4, FAKE, ws, FAKE, FAKE, FAKE, None) == 1
+    assert lib.tf_ring_attn(FAKE, 1, 8, FAKE, FAKE, 100, 2, 64, FAKE, 1, None, 0.1, 64, 4, FAKE, ws - 1, FAKE, FAKE,
+                            FAKE, None) == 7
+    seg = np.array([[0, 4, 3, 0, 1]], np.int32)  # more rows than keys
+    assert lib.tf_paged_attn_prompt(FAKE, 4, 8, FAKE, FAKE, 4, 16, 2, 64, FAKE, 1, seg.ctypes.data_as(ctypes.c_void_p),
+                                    0.1, FAKE, 1, None, FAKE, None) == 1
