@@ -1,0 +1,561 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV-cache segment attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--only decode]
+
+Headline: multi-stream decode (16 one-row streams, 32/8 heads, head dim 128,
+pages of 32 in a shuffled 8,192-page pool, 512-key partials + merge).  A step
+is one decode pass over that batch: the split-KV partial kernel and the merge.
+value = KV bytes a step reads (every visible key once per kv-head) / step time,
+in GB/s, with inputs resident in HBM and L2 flushed (a 256 MiB write) before
+every timed step.  At N > 1 every rank runs its own replica of the batch
+(independent streams, no collective on the data path) and value = all ranks'
+bytes / the slowest rank's time ("weak" scaling).
+
+Also reported (N = 1): the shared verify round (decode + merge + argmax), the
+drafter ring, the 15,000-token prompt (TFLOP/s) and the 128,000-wide argmax
+(rows/s), each with its own roofline; an end-to-end number through the public
+API with host buffers; and the float64 oracle timed on the host cores.
+
+--impl reference times the float64 oracle (the only reference there is) on
+the same workload, metric and unit, a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "paged attn decode KV GB/s (% HBM peak); prompt attn TFLOP/s; argmax rows/s"
+WORKLOAD = ("multi-stream decode: 16 streams x 1 row, 32 q / 8 kv heads, head dim 128, pages of 32 in a shuffled "
+            "8,192-page pool, contexts U{1024..8192}, 512-key split-KV partials + merge, fp32 out")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+# ----------------------------------------------------------------------------- args / env
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--only", default="", help="comma list: decode,verify,ring,prompt,argmax,e2e,cpu")
+    ap.add_argument("--secondary-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def want(args, what):
+    return not args.only or what in args.only.split(",")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {**FALLBACK_PEAKS, "source": "fallback"}
+
+
+def load_traffic():
+    """ncu DRAM bytes per launch recorded in profiles/ncu_traffic.json, valid
+    only while the kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    out = {}
+    for key, rec in d.items():
+        src = os.path.join(ROOT, rec["source"])
+        try:
+            sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        except OSError:
+            continue
+        out[key] = rec["dram_bytes_per_launch"] if sha == rec["source_sha256"] else None
+    return out
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while timing runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, n = [], None, set(), 0
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            n += 1
+            for name, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s in sm if smax and s > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def clocks_bad(c):
+    if any(r in BAD_REASONS for r in c.get("reasons", [])):
+        return True
+    if c.get("sm_mhz") and c.get("sm_max_mhz") and c["sm_mhz"] < 0.5 * c["sm_max_mhz"] and not c.get("reasons"):
+        return True
+    return False
+
+
+# ----------------------------------------------------------------------------- device helpers
+
+def to_dev(a, dev):
+    import torch
+
+    a = np.ascontiguousarray(a)
+    return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+
+
+class DecodeRun:
+    """Device buffers and the two launches of one decode pass."""
+
+    def __init__(self, b, dev, logits=None):
+        import torch
+
+        self.b = b
+        rows, hq, d = b.q.shape
+        self.q, self.kp, self.vp = to_dev(b.q, dev), to_dev(b.k_pool, dev), to_dev(b.v_pool, dev)
+        self.pt, self.segs = to_dev(b.page_table, dev), to_dev(b.segs, dev)
+        c = b.n_splits_max
+        self.po = torch.empty((rows, hq, c, d), device=dev)
+        self.pm = torch.empty((rows, hq, c), device=dev)
+        self.pl = torch.empty((rows, hq, c), device=dev)
+        self.pf = torch.empty((rows, hq, c), dtype=torch.uint8, device=dev)
+        self.out = torch.empty((rows, hq, d), device=dev)
+        self.fl = torch.empty((rows, hq), dtype=torch.uint8, device=dev)
+        self.st = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.logits = to_dev(logits, dev) if logits is not None else None
+        if logits is not None:
+            self.ids = torch.empty(logits.shape[0], dtype=torch.int32, device=dev)
+            self.afl = torch.empty(logits.shape[0], dtype=torch.uint8, device=dev)
+
+    def partial(self):
+        import paged_kv_cache_segment_b200 as tf
+
+        b = self.b
+        tf.tf_paged_attn_decode(self.q, self.kp, self.vp, self.pt, self.segs, scale=b.scale, split_keys=b.split_keys,
+                                n_splits_max=b.n_splits_max, part_o=self.po, part_m=self.pm, part_l=self.pl,
+                                part_flag=self.pf, status=self.st, segs_host=b.segs)
+
+    def merge(self):
+        import paged_kv_cache_segment_b200 as tf
+
+        tf.tf_attn_merge(self.po, self.pm, self.pl, self.pf, self.out, self.fl)
+
+    def argmax(self):
+        import paged_kv_cache_segment_b200 as tf
+
+        tf.tf_argmax_rows(self.logits, self.ids, self.afl)
+
+
+def timed_steps(launches, steps, flush):
+    """Run `steps` steps; before each one flush L2 (untimed), then time each
+    launch of the step with CUDA events on the current stream.  Returns the
+    per-launch total milliseconds and the step total."""
+    import torch
+
+    n = len(launches)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    for s in range(steps):
+        flush.zero_()
+        evs[s][0].record()
+        for k, fn in enumerate(launches):
+            fn()
+            evs[s][k + 1].record()
+    torch.cuda.synchronize()
+    per = [0.0] * n
+    total = 0.0
+    for s in range(steps):
+        for k in range(n):
+            per[k] += evs[s][k].elapsed_time(evs[s][k + 1])
+        total += evs[s][0].elapsed_time(evs[s][n])
+    return per, total
+
+
+def roofline(bound, achieved, peak, unit, traffic=None):
+    return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic}
+
+
+# ----------------------------------------------------------------------------- the native arm
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_cache_segment_b200 import workloads as wl
+    import paged_kv_cache_segment_b200 as tf
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    tf.load()
+    peaks = load_peaks()
+    traffic = load_traffic()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # -------------------------------------------------------------- headline: decode
+    b = wl.multi_stream_decode(2)
+    kv_bytes = b.kv_bytes()
+    run = DecodeRun(b, dev)
+    for _ in range(max(3, args.warmup)):
+        run.partial()
+        run.merge()
+    barrier()
+    sampler = ClockSampler(local)
+    result = None
+    for attempt in range(2):
+        sampler.start()
+        barrier()
+        per, total = timed_steps([run.partial, run.merge], args.steps, flush)
+        barrier()
+        clocks = sampler.stop()
+        if not clocks_bad(clocks) or attempt == 1:
+            break
+    total_max = max_over_ranks(total)
+    part_ms = per[0] / args.steps
+    ms_step = total_max / args.steps
+    assert int(run.st.item()) == 0, "device status set during the decode bench"
+    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    achieved = kv_bytes / (part_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded PCG64; bf16 ~N(0,1))",
+        "config": {"workload": WORKLOAD, "streams": 16, "kv_bytes_per_step": kv_bytes,
+                   "parallelism": f"replicas x{world}", "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": roofline("hbm", achieved, peaks["hbm_gbs"], "GB/s", traffic.get("decode_partial_cfg2")),
+        "kernels": {"decode_partial_ms": round(part_ms, 5), "merge_ms": round(per[1] / args.steps, 5)},
+        "peaks_source": peaks["source"],
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    result["roofline"]["kernel"] = "attn_partial_kernel<128, paged>"
+    result["roofline"]["frac_of"] = "measured" if peaks["source"] == "measured" else "fallback"
+    result["roofline"]["frac_of_8tbs"] = round(achieved / 8000.0, 4)
+
+    # -------------------------------------------------------------- e2e through the public API, host buffers
+    if want(args, "e2e"):
+        result["e2e"] = e2e_decode(b, run, flush, min(args.steps, 500), barrier, max_over_ranks, world)
+
+    # -------------------------------------------------------------- secondary workloads (N = 1 only)
+    if world == 1:
+        sec = {}
+        ks = args.secondary_steps
+        if want(args, "verify") or want(args, "argmax"):
+            sec.update(bench_verify(wl, dev, flush, ks, peaks, traffic))
+        if want(args, "ring"):
+            sec["ring"] = bench_ring(wl, tf, dev, flush, ks, peaks)
+        if want(args, "prompt"):
+            sec["prompt"] = bench_prompt(wl, tf, dev, flush, max(3, ks // 4), peaks)
+        result["secondary"] = sec
+        result["gpu_launches_secondary"] = sum(v.get("launches", 0) for v in sec.values())
+    if rank == 0 and world == 1 and want(args, "cpu"):
+        result["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def e2e_decode(b, run, flush, steps, barrier, max_over_ranks, world):
+    """The decode step through the public API with HOST inputs and outputs:
+    pinned q / segment table / page table copied in, partials + merge, the
+    output and flags copied back, every step inside the timed region.  The KV
+    pool is the cache: it stays resident on the device."""
+    import torch
+
+    import paged_kv_cache_segment_b200 as tf
+
+    q_h = torch.from_numpy(b.q.view(np.int16)).pin_memory()
+    seg_h = torch.from_numpy(b.segs).pin_memory()
+    pt_h = torch.from_numpy(b.page_table).pin_memory()
+    out_h = torch.empty(tuple(run.out.shape), dtype=torch.float32).pin_memory()
+    fl_h = torch.empty(tuple(run.fl.shape), dtype=torch.uint8).pin_memory()
+    h2d = q_h.numel() * 2 + seg_h.numel() * 4 + pt_h.numel() * 4
+    d2h = out_h.numel() * 4 + fl_h.numel()
+
+    def step():
+        run.q.copy_(q_h, non_blocking=True)
+        run.segs.copy_(seg_h, non_blocking=True)
+        run.pt.copy_(pt_h, non_blocking=True)
+        tf.tf_paged_attn_decode(run.q, run.kp, run.vp, run.pt, run.segs, scale=b.scale, split_keys=b.split_keys,
+                                n_splits_max=b.n_splits_max, part_o=run.po, part_m=run.pm, part_l=run.pl,
+                                part_flag=run.pf, status=run.st, segs_host=b.segs)
+        tf.tf_attn_merge(run.po, run.pm, run.pl, run.pf, run.out, run.fl)
+        out_h.copy_(run.out, non_blocking=True)
+        fl_h.copy_(run.fl, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    barrier()
+    _, total = timed_steps([step], steps, flush)
+    barrier()
+    total = max_over_ranks(total)
+    ms = total / steps
+    return {"value": round(world * b.kv_bytes() / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 5),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "path": "binding tf_paged_attn_decode + tf_attn_merge, pinned host buffers"}
+
+
+def bench_verify(wl, dev, flush, steps, peaks, traffic):
+    b = wl.shared_verify(3)
+    rows = b.n_rows_total
+    logits = wl.verify_logits(3, rows)
+    run = DecodeRun(b, dev, logits)
+    for _ in range(3):
+        run.partial()
+        run.merge()
+        run.argmax()
+    per, total = timed_steps([run.partial, run.merge, run.argmax], steps, flush)
+    kv = b.kv_bytes()
+    pms, mms, ams = per[0] / steps, per[1] / steps, per[2] / steps
+    flops = 4 * b.head_dim * sum(int(s[1]) * b.n_q_heads * (int(s[2]) - int(s[1]) + 1) + b.n_q_heads *
+                                 int(s[1]) * (int(s[1]) - 1) // 2 for s in b.segs)
+    arg_bytes = rows * 128000 * 2
+    out = {
+        "verify": {"workload": "shared verify: 8 streams x U{1..16} rows, 16/2 heads, D256, P32, contexts "
+                               "U{2048..16384}, 1024-key partials + merge", "rows": rows,
+                   "kv_gbs": round(kv / (pms + mms) / 1e6, 2), "ms_per_step": round((pms + mms), 5),
+                   "tflops": round(flops / (pms * 1e-3) / 1e12, 2),
+                   "roofline": roofline("hbm", kv / (pms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                                        traffic.get("decode_partial_cfg3")),
+                   "launches": 2 * steps},
+        "argmax": {"workload": f"{rows} rows x 128,000 bf16 ~N(0,3), ties in ~1/4 of rows",
+                   "rows_per_s": round(rows / (ams * 1e-3), 1), "ms": round(ams, 5),
+                   "roofline": roofline("hbm", arg_bytes / (ams * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                                        traffic.get("argmax_cfg3")),
+                   "launches": steps},
+    }
+    assert int(run.st.item()) == 0
+    return out
+
+
+def bench_ring(wl, tf, dev, flush, steps, peaks):
+    import torch
+
+    from paged_kv_cache_segment_b200 import binding
+
+    b = wl.drafter_ring(5)
+    n = len(b.rsegs)
+    hq, d = b.n_q_heads, b.head_dim
+    q, rk, rv = to_dev(b.q, dev), to_dev(b.ring_k, dev), to_dev(b.ring_v, dev)
+    rs = binding.rsegs_to_device(b.rsegs, dev)
+    ws = torch.empty(tf.tf_ring_workspace_bytes(n, hq, d, b.n_splits_max), dtype=torch.uint8, device=dev)
+    out = torch.empty((n, hq, d), device=dev)
+    fl = torch.empty((n, hq), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step():
+        tf.tf_ring_attn(q, rk, rv, rs, scale=b.scale, split_slots=b.split_slots, n_splits_max=b.n_splits_max,
+                        workspace=ws, out=out, flags=fl, status=st, rsegs_host=b.rsegs)
+
+    for _ in range(3):
+        step()
+    per, total = timed_steps([step], steps, flush)
+    ms = total / steps
+    kv = b.kv_bytes()
+    assert int(st.item()) == 0
+    return {"workload": "drafter ring: 17 rows, rings of 4,200 slots, random heads, U{1000..4200} valid, 16/2 heads, "
+                        "D256, 256-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
+            "ms_per_step": round(ms, 5), "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
+            "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"), "launches": 2 * steps}
+
+
+def bench_prompt(wl, tf, dev, flush, steps, peaks):
+    import torch
+
+    b, spans = wl.long_prompt(4)
+    rows, hq, d = b.q.shape
+    q, kp, vp, pt = to_dev(b.q, dev), to_dev(b.k_pool, dev), to_dev(b.v_pool, dev), to_dev(b.page_table, dev)
+    out = torch.empty((rows, hq, d), dtype=torch.bfloat16, device=dev)
+    fl = torch.empty((rows, hq), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    segs = [wl.prompt_chunk_seg(b, r0, r1) for r0, r1 in spans]
+
+    def step():
+        for sg in segs:
+            tf.tf_paged_attn_prompt(q, kp, vp, pt, sg, scale=b.scale, out=out, flags=fl, status=st)
+
+    step()
+    per, total = timed_steps([step], steps, flush)
+    ms = total / steps
+    n = rows
+    flops = 4 * d * hq * n * (n + 1) // 2
+    assert int(st.item()) == 0
+    tfl = flops / (ms * 1e-3) / 1e12
+    return {"workload": "long causal prompt: 15,000 tokens in 2,048-row chunks, 16/4 heads, D256, P32, 469 shuffled "
+                        "pages, bf16 out", "tflops": round(tfl, 2), "ms_per_step": round(ms, 4),
+            "algorithmic_flops": flops,
+            "roofline": roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s"), "launches": len(segs) * steps}
+
+
+def cpu_baseline(b, seconds):
+    """The float64 oracle, as it stands, on this host's cores: whole passes of
+    the decode workload repeated for about `seconds`."""
+    import oracle
+
+    orc = oracle.get()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        orc.paged_attn(b.q, b.k_pool, b.v_pool, b.page_table, b.segs, b.scale)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": round(reps * b.kv_bytes() / el / 1e9, 4), "unit": "GB/s", "cores": orc.num_threads(),
+            "kind": "oracle", "sample": f"{reps} whole passes of the 16-stream decode batch in {el:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- the reference arm (the oracle)
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from paged_kv_cache_segment_b200 import workloads as wl
+
+    orc = oracle.get()
+    b = wl.multi_stream_decode(2)
+    hq, hkv = b.n_q_heads, b.n_kv_heads
+    group = hq // hkv
+    units = [(s, g) for s in range(len(b.segs)) for g in range(hkv)]
+    # one (stream, kv-head) unit a step; every q-head of the group is computed
+    sel_cache = {}
+
+    def step(k):
+        s, g = units[k % len(units)]
+        if (s, g) not in sel_cache:
+            sel = np.zeros((b.n_rows_total, hq), np.uint8)
+            sel[b.segs[s][0], g * group:(g + 1) * group] = 1
+            sel_cache[(s, g)] = sel
+        seg = b.segs[s:s + 1]
+        orc.paged_attn(b.q, b.k_pool, b.v_pool, b.page_table, seg, b.scale, sel=sel_cache[(s, g)])
+        return int(b.segs[s][2]) * b.head_dim * 2 * 2
+
+    budget = 150.0
+    for k in range(args.warmup):
+        step(k)
+    t0 = time.perf_counter()
+    nbytes = 0
+    done = 0
+    for k in range(args.steps):
+        nbytes += step(k)
+        done += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    el = time.perf_counter() - t0
+    v = nbytes / el / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": done, "warmup": args.warmup, "ms_per_step": round(el / max(done, 1) * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": "one (stream, kv-head) unit of the batch a step, all its q-heads"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": orc.num_threads(), "kind": "oracle",
+                         "sample": f"{done} (stream, kv-head) units in {el:.1f} s"},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()
