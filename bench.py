@@ -241,6 +241,24 @@ def timed_steps(launches, steps, flush):
     return per, total
 
 
+def reduce_max(x: float, device, world: int) -> float:
+    """The largest value of x over all ranks (every rank calls it, in the
+    same order); the slowest rank's time is the job's time."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job GB/s: every rank's replica bytes over the slowest rank's time."""
+    return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
+
+
 def roofline(bound, achieved, peak, unit, traffic=None):
     return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic}
@@ -276,11 +294,7 @@ def run_native(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dev, world)
 
     # -------------------------------------------------------------- headline: decode
     b = wl.multi_stream_decode(2)
@@ -304,7 +318,7 @@ def run_native(args):
     part_ms = per[0] / args.steps
     ms_step = total_max / args.steps
     assert int(run.st.item()) == 0, "device status set during the decode bench"
-    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(kv_bytes, world, ms_step)
     achieved = kv_bytes / (part_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
