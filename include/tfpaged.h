@@ -202,6 +202,39 @@ TF_API tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_h
 TF_API size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max);
 
 /*
+ * tf_ring_attn for callers that cannot allocate device memory.  The pages
+ * have no counterpart of this call; it exists for this library's users.
+ *
+ * Some callers have no workspace to give: a serving engine that hands all
+ * device memory to its KV pool at start-up and keeps no allocator on the
+ * decode path, or a host framework that calls this library from a plugin
+ * hook where cudaMalloc, and the device-wide synchronization it can imply,
+ * is not allowed.  This call keeps the partials in a scratch array that is
+ * part of the library's own device image: TF_RING_NOALLOC_SCRATCH_BYTES
+ * bytes that every GPU which loads the library holds until the process
+ * exits.  Arguments and results are tf_ring_attn's, less the workspace.
+ *
+ *  - Sizes whose tf_ring_workspace_bytes(n_segs, n_q_heads, head_dim,
+ *    n_splits_max) exceeds TF_RING_NOALLOC_SCRATCH_BYTES are refused with
+ *    TF_ERR_WORKSPACE before anything is launched.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture.  Nothing is allocated by this library, then or later.
+ *  - Every call on a device shares the one scratch array and leaves its
+ *    partials there.  Nothing in it needs to start at zero (every partial
+ *    the merge reads is written first by the same call), but two calls whose
+ *    kernels overlap on the GPU (different streams, no ordering between them)
+ *    race on it: order them, or use tf_ring_attn with separate workspaces.
+ */
+#define TF_RING_NOALLOC_SCRATCH_BYTES (8u << 20)
+TF_API tf_status tf_ring_attn_noalloc(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *ring_k,
+                                      const void *ring_v, int64_t ring_slots_total, int32_t n_kv_heads,
+                                      int32_t head_dim, const tf_ring_seg *rsegs, int32_t n_segs,
+                                      const tf_ring_seg *rsegs_host, float scale, int32_t split_slots,
+                                      int32_t n_splits_max, float *out, uint8_t *flags, uint32_t *status,
+                                      tf_stream_t stream);
+
+/*
  * Greedy row argmax (lfm2_argmax of #1503, commit list): for each of n_rows
  * rows of n_cols bf16 logits (row stride ld elements), ids[r] = the lowest
  * column holding the row's largest value, values compared as real numbers

@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     tf_paged_attn_decode,
     tf_paged_attn_prompt,
     tf_ring_attn,
+    tf_ring_attn_noalloc,
     tf_ring_workspace_bytes,
     tf_status_str,
 )

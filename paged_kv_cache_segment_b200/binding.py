@@ -25,7 +25,9 @@ TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS = 1, 2, 4, 8
 TF_OUT_F32, TF_OUT_BF16 = 0, 1
 
 EXPORTS = ("tf_paged_attn_decode", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
-           "tf_ring_workspace_bytes", "tf_argmax_rows", "tf_status_str", "tf_abi_version")
+           "tf_ring_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_status_str", "tf_abi_version")
+# bytes of the scratch array tf_ring_attn_noalloc keeps in the library's device image
+TF_RING_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 SEG_DTYPE = np.dtype([("q_row", "<i4"), ("n_rows", "<i4"), ("n_keys", "<i4"), ("pt_base", "<i4"), ("n_pages", "<i4")])
 RING_SEG_DTYPE = np.dtype(
@@ -56,13 +58,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_attn_merge.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P]
     lib.tf_paged_attn_prompt.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, f32, P, i32, P, P, P]
     lib.tf_ring_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, f32, i32, i32, P, sz, P, P, P, P]
+    lib.tf_ring_attn_noalloc.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, f32, i32, i32, P, P, P, P]
     lib.tf_ring_workspace_bytes.argtypes = [i32, i32, i32, i32]
     lib.tf_ring_workspace_bytes.restype = sz
     lib.tf_argmax_rows.argtypes = [P, i32, i32, i64, P, P, P]
     lib.tf_status_str.argtypes = [ctypes.c_int]
     lib.tf_status_str.restype = ctypes.c_char_p
     lib.tf_abi_version.restype = ctypes.c_int32
-    for name in ("tf_paged_attn_decode", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn", "tf_argmax_rows"):
+    for name in ("tf_paged_attn_decode", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
+                 "tf_ring_attn_noalloc", "tf_argmax_rows"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -189,6 +193,27 @@ def tf_ring_attn(q, ring_k, ring_v, rsegs, *, scale, split_slots, n_splits_max, 
                           _dev(out, "out", (torch.float32,)), _dev(flags, "flags", (torch.uint8,)),
                           _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
     _check("tf_ring_attn", rc)
+
+
+def tf_ring_attn_noalloc(q, ring_k, ring_v, rsegs, *, scale, split_slots, n_splits_max, out, flags, status,
+                         rsegs_host=None, stream=None):
+    """tf_ring_attn without a workspace, for callers that cannot allocate
+    device memory: the partials go to a scratch array built into the
+    library (TF_RING_NOALLOC_SCRATCH_BYTES bytes a GPU, held until exit).
+    All calls on a device share it, so calls must not overlap on the GPU;
+    the first call on a device should come before any stream capture."""
+    lib = load()
+    rows, hq, d = q.shape
+    slots, hkv, d2 = ring_k.shape
+    n_segs = rsegs.numel() // RING_SEG_DTYPE.itemsize
+    rh = as_rsegs_np(rsegs_host) if rsegs_host is not None else None
+    rc = lib.tf_ring_attn_noalloc(_dev(q, "q", BF16), rows, hq, _dev(ring_k, "ring_k", BF16),
+                                  _dev(ring_v, "ring_v", BF16), slots, hkv, d,
+                                  _dev(rsegs, "rsegs", (torch.uint8, torch.int8)), n_segs, _host_ptr(rh),
+                                  float(scale), int(split_slots), int(n_splits_max),
+                                  _dev(out, "out", (torch.float32,)), _dev(flags, "flags", (torch.uint8,)),
+                                  _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
+    _check("tf_ring_attn_noalloc", rc)
 
 
 def tf_argmax_rows(logits, ids, flags, *, n_cols=None, stream=None):
