@@ -84,6 +84,7 @@ typedef enum {
 #define TF_DEV_PAST_PAGES 0x2u /* n_keys > n_pages * page_size (the pages' PastPages refusal) */
 #define TF_DEV_BAD_PAGE 0x4u   /* a page id outside [0, n_pages of the pool) */
 #define TF_DEV_SPLITS 0x8u     /* a stream needs more partials than n_splits_max */
+#define TF_DEV_TIMEOUT 0x10u   /* a bounded wait inside a kernel gave up; that CTA's outputs are flagged */
 
 /* One stream's entry in the segment table (device array, int32 fields). */
 typedef struct {

@@ -163,6 +163,27 @@ tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_
     const int64_t n_qgroups = ((int64_t)max_rows * group + 63) / 64;
     if (n_qgroups * n_kv_heads > 65535) return TF_ERR_UNSUPPORTED;
 
+    if (prompt_tc_supported(head_dim, group, page_size)) {
+        PromptTcParams t{};
+        t.q_row = seg_host->q_row;
+        t.n_rows = seg_host->n_rows;
+        t.n_keys = seg_host->n_keys;
+        t.pt_base = seg_host->pt_base;
+        t.n_pg = seg_host->n_pages;
+        t.page_table = page_table;
+        t.n_pages = n_pages;
+        t.log2_page = lp;
+        t.hq = n_q_heads;
+        t.hkv = n_kv_heads;
+        t.group = group;
+        t.n_rows_total = n_rows_total;
+        t.scale_log2 = scale * 1.4426950408889634f;
+        t.out = out;
+        t.out_bf16 = out_dtype == TF_OUT_BF16;
+        t.out_flags = flags;
+        t.status = status;
+        return cuda_status(launch_prompt_tc(t, head_dim, q, k_pool, v_pool, reinterpret_cast<cudaStream_t>(stream)));
+    }
     AttnParams p{};
     p.q = static_cast<const uint16_t *>(q);
     p.n_rows_total = n_rows_total;

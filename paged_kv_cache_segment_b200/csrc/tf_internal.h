@@ -47,6 +47,18 @@ struct MergeParams {
     uint8_t *flags;
 };
 
+// Parameters of the tensor-core prompt kernel (one stream's chunk).
+struct PromptTcParams {
+    int q_row, n_rows, n_keys, pt_base, n_pg;  // the chunk's segment
+    const int32_t *page_table;
+    int n_pages, log2_page, hq, hkv, group, n_rows_total;
+    float scale_log2;
+    void *out;
+    int out_bf16;
+    uint8_t *out_flags;
+    uint32_t *status;
+};
+
 struct ArgmaxParams {
     const uint16_t *logits;
     int n_rows, n_cols;
@@ -59,6 +71,9 @@ cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bo
                                 cudaStream_t st);
 cudaError_t launch_merge(const MergeParams &p, int head_dim, bool ring, cudaStream_t st);
 cudaError_t launch_argmax(const ArgmaxParams &p, bool vec, cudaStream_t st);
+bool prompt_tc_supported(int head_dim, int group, int page_size);
+cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *q, const void *k, const void *v,
+                             cudaStream_t st);
 
 constexpr int kArgmaxCluster = 8;
 

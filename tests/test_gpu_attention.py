@@ -389,3 +389,37 @@ def test_long_prompt_sampled_rows(orc):
     np.testing.assert_array_equal(r["flags"], np.zeros_like(r["flags"]))
     err = np.abs(r["out"][sel] - ref[sel])
     assert (err <= bf16_ulp(ref[sel]) + 1e-5).all(), f"bf16 prompt beyond one ulp: {err.max()}"
+
+
+@pytest.mark.parametrize("hq,hkv,d,p,n,chunk", [(16, 4, 256, 32, 700, 256), (8, 8, 64, 16, 300, 100),
+                                                (8, 2, 128, 64, 513, 200), (4, 1, 128, 256, 1000, 384),
+                                                (6, 2, 64, 16, 200, 64), (32, 4, 128, 32, 260, 260),
+                                                (16, 2, 256, 8, 150, 150)])
+def test_prompt_shapes(orc, hq, hkv, d, p, n, chunk):
+    """Prompt chunks at several head counts, head dims and page sizes (G = 3
+    takes the mma.sync path, every other shape the tensor-memory one)."""
+    b = wl.make_paged_batch(n + d + p, rows=[n], keys=[n], n_q_heads=hq, n_kv_heads=hkv, head_dim=d, page_size=p,
+                            unused="nan", split_keys=0, n_splits_max=1)
+    spans = [(a, min(a + chunk, n)) for a in range(0, n, chunk)]
+    r = run_prompt_chunks(b, spans, out_dtype=torch.float32)
+    assert r["status"] == 0
+    ref, rf = orc.paged_attn(b.q, b.k_pool, b.v_pool, b.page_table, b.segs, b.scale)
+    compare_attn(r["out"], r["flags"], ref, rf, what=f"prompt {hq}/{hkv} D{d} P{p}")
+
+
+def test_prompt_nonfinite_flags(orc):
+    """Inf in an early key (seen by rows 3 on), NaN in a value only the chunk's
+    last rows see, -Inf in one q element: flags equal the oracle's."""
+    n = 400
+    b = wl.make_paged_batch(77, rows=[n], keys=[n], n_q_heads=16, n_kv_heads=4, head_dim=256, page_size=32,
+                            unused="nan", split_keys=0, n_splits_max=1)
+    pt = b.page_table
+    b.k_pool[pt[3 // 32], 1, 3 % 32, 7] = wl.BF16_POS_INF
+    b.v_pool[pt[395 // 32], 2, 395 % 32, 100] = wl.BF16_NAN
+    b.q[250, 13, 0] = wl.BF16_NEG_INF
+    spans = [(0, 200), (200, 400)]
+    r = run_prompt_chunks(b, spans, out_dtype=torch.float32)
+    ref, rf = orc.paged_attn(b.q, b.k_pool, b.v_pool, b.page_table, b.segs, b.scale)
+    assert rf[3:, 4:8].all() and not rf[:3, 4:8].any()  # key 3 is seen by rows 3..
+    assert rf[395:, 8:12].all() and not rf[:395, 8:12].any() and rf[250, 13]
+    compare_attn(r["out"], r["flags"], ref, rf, what="prompt flags")
