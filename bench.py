@@ -7,8 +7,8 @@ Headline: multi-stream decode (16 one-row streams, 32/8 heads, head dim 128,
 pages of 32 in a shuffled 8,192-page pool, 512-key partials + merge).  A step
 is one decode pass over that batch: the split-KV partial kernel and the merge.
 value = KV bytes a step reads (every visible key once per kv-head) / step time,
-in GB/s, with inputs resident in HBM and L2 flushed (a 256 MiB write) before
-every timed step.  At N > 1 every rank runs its own replica of the batch
+in GB/s, with inputs resident in HBM; three copies of the batch rotate between
+steps (906 MB of KV, over seven times the L2), so no step finds its data in L2.  At N > 1 every rank runs its own replica of the batch
 (independent streams, no collective on the data path) and value = all ranks'
 bytes / the slowest rank's time ("weak" scaling).
 
@@ -42,7 +42,6 @@ METRIC = "paged attn decode KV GB/s (% HBM peak); prompt attn TFLOP/s; argmax ro
 WORKLOAD = ("multi-stream decode: 16 streams x 1 row, 32 q / 8 kv heads, head dim 128, pages of 32 in a shuffled "
             "8,192-page pool, contexts U{1024..8192}, 512-key split-KV partials + merge, fp32 out")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-L2_FLUSH_BYTES = 256 << 20
 BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -176,15 +175,19 @@ def to_dev(a, dev):
 
 
 class DecodeRun:
-    """Device buffers and the two launches of one decode pass."""
+    """Device buffers and the launches of one decode pass.  `copies` sets of
+    the inputs live at different addresses; step k reads set k % copies, so
+    with their total above the L2 size no step finds its data in L2."""
 
-    def __init__(self, b, dev, logits=None):
+    def __init__(self, b, dev, logits=None, copies=3):
         import torch
 
         self.b = b
         rows, hq, d = b.q.shape
-        self.q, self.kp, self.vp = to_dev(b.q, dev), to_dev(b.k_pool, dev), to_dev(b.v_pool, dev)
-        self.pt, self.segs = to_dev(b.page_table, dev), to_dev(b.segs, dev)
+        self.sets = [dict(q=to_dev(b.q, dev), kp=to_dev(b.k_pool, dev), vp=to_dev(b.v_pool, dev),
+                          pt=to_dev(b.page_table, dev), segs=to_dev(b.segs, dev),
+                          logits=to_dev(logits, dev) if logits is not None else None)
+                     for _ in range(copies)]
         c = b.n_splits_max
         self.po = torch.empty((rows, hq, c, d), device=dev)
         self.pm = torch.empty((rows, hq, c), device=dev)
@@ -193,43 +196,42 @@ class DecodeRun:
         self.out = torch.empty((rows, hq, d), device=dev)
         self.fl = torch.empty((rows, hq), dtype=torch.uint8, device=dev)
         self.st = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.logits = to_dev(logits, dev) if logits is not None else None
         if logits is not None:
             self.ids = torch.empty(logits.shape[0], dtype=torch.int32, device=dev)
             self.afl = torch.empty(logits.shape[0], dtype=torch.uint8, device=dev)
 
-    def partial(self):
+    def partial(self, k=0):
         import paged_kv_cache_segment_b200 as tf
 
-        b = self.b
-        tf.tf_paged_attn_decode(self.q, self.kp, self.vp, self.pt, self.segs, scale=b.scale, split_keys=b.split_keys,
-                                n_splits_max=b.n_splits_max, part_o=self.po, part_m=self.pm, part_l=self.pl,
-                                part_flag=self.pf, status=self.st, segs_host=b.segs)
+        b, x = self.b, self.sets[k % len(self.sets)]
+        tf.tf_paged_attn_decode(x["q"], x["kp"], x["vp"], x["pt"], x["segs"], scale=b.scale,
+                                split_keys=b.split_keys, n_splits_max=b.n_splits_max, part_o=self.po,
+                                part_m=self.pm, part_l=self.pl, part_flag=self.pf, status=self.st,
+                                segs_host=b.segs)
 
-    def merge(self):
+    def merge(self, k=0):
         import paged_kv_cache_segment_b200 as tf
 
         tf.tf_attn_merge(self.po, self.pm, self.pl, self.pf, self.out, self.fl)
 
-    def argmax(self):
+    def argmax(self, k=0):
         import paged_kv_cache_segment_b200 as tf
 
-        tf.tf_argmax_rows(self.logits, self.ids, self.afl)
+        tf.tf_argmax_rows(self.sets[k % len(self.sets)]["logits"], self.ids, self.afl)
 
 
-def timed_steps(launches, steps, flush):
-    """Run `steps` steps; before each one flush L2 (untimed), then time each
-    launch of the step with CUDA events on the current stream.  Returns the
-    per-launch total milliseconds and the step total."""
+def timed_steps(launches, steps):
+    """Run `steps` steps, timing each launch of a step with CUDA events on the
+    current stream.  Each launch gets the step index (it picks the input copy).
+    Returns the per-launch total milliseconds and the step total."""
     import torch
 
     n = len(launches)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
     for s in range(steps):
-        flush.zero_()
         evs[s][0].record()
         for k, fn in enumerate(launches):
-            fn()
+            fn(s)
             evs[s][k + 1].record()
     torch.cuda.synchronize()
     per = [0.0] * n
@@ -286,7 +288,6 @@ def run_native(args):
     tf.load()
     peaks = load_peaks()
     traffic = load_traffic()
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def barrier():
         if world > 1:
@@ -309,7 +310,7 @@ def run_native(args):
     for attempt in range(2):
         sampler.start()
         barrier()
-        per, total = timed_steps([run.partial, run.merge], args.steps, flush)
+        per, total = timed_steps([run.partial, run.merge], args.steps)
         barrier()
         clocks = sampler.stop()
         if not clocks_bad(clocks) or attempt == 1:
@@ -325,31 +326,32 @@ def run_native(args):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded PCG64; bf16 ~N(0,1))",
         "config": {"workload": WORKLOAD, "streams": 16, "kv_bytes_per_step": kv_bytes,
-                   "parallelism": f"replicas x{world}", "l2": "flushed before every timed step (256 MiB write)"},
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: 3 rotating copies of the batch (906 MB of KV), step k reads copy k % 3"},
         "roofline": roofline("hbm", achieved, peaks["hbm_gbs"], "GB/s", traffic.get("decode_partial_cfg2")),
         "kernels": {"decode_partial_ms": round(part_ms, 5), "merge_ms": round(per[1] / args.steps, 5)},
         "peaks_source": peaks["source"],
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
-    result["roofline"]["kernel"] = "attn_partial_kernel<128, paged>"
+    result["roofline"]["kernel"] = "decode_ws_kernel<128, paged>"
     result["roofline"]["frac_of"] = "measured" if peaks["source"] == "measured" else "fallback"
     result["roofline"]["frac_of_8tbs"] = round(achieved / 8000.0, 4)
 
     # -------------------------------------------------------------- e2e through the public API, host buffers
     if want(args, "e2e"):
-        result["e2e"] = e2e_decode(b, run, flush, min(args.steps, 500), barrier, max_over_ranks, world)
+        result["e2e"] = e2e_decode(b, run, min(args.steps, 500), barrier, max_over_ranks, world)
 
     # -------------------------------------------------------------- secondary workloads (N = 1 only)
     if world == 1:
         sec = {}
         ks = args.secondary_steps
         if want(args, "verify") or want(args, "argmax"):
-            sec.update(bench_verify(wl, dev, flush, ks, peaks, traffic))
+            sec.update(bench_verify(wl, dev, ks, peaks, traffic))
         if want(args, "ring"):
-            sec["ring"] = bench_ring(wl, tf, dev, flush, ks, peaks)
+            sec["ring"] = bench_ring(wl, tf, dev, ks, peaks)
         if want(args, "prompt"):
-            sec["prompt"] = bench_prompt(wl, tf, dev, flush, max(3, ks // 4), peaks)
+            sec["prompt"] = bench_prompt(wl, tf, dev, max(3, ks // 4), peaks)
         result["secondary"] = sec
         result["gpu_launches_secondary"] = sum(v.get("launches", 0) for v in sec.values())
     if rank == 0 and world == 1 and want(args, "cpu"):
@@ -361,11 +363,11 @@ def run_native(args):
         print(json.dumps(result))
 
 
-def e2e_decode(b, run, flush, steps, barrier, max_over_ranks, world):
+def e2e_decode(b, run, steps, barrier, max_over_ranks, world):
     """The decode step through the public API with HOST inputs and outputs:
     pinned q / segment table / page table copied in, partials + merge, the
     output and flags copied back, every step inside the timed region.  The KV
-    pool is the cache: it stays resident on the device."""
+    pool is the cache: it stays resident on the device (rotating copies)."""
     import torch
 
     import paged_kv_cache_segment_b200 as tf
@@ -378,21 +380,22 @@ def e2e_decode(b, run, flush, steps, barrier, max_over_ranks, world):
     h2d = q_h.numel() * 2 + seg_h.numel() * 4 + pt_h.numel() * 4
     d2h = out_h.numel() * 4 + fl_h.numel()
 
-    def step():
-        run.q.copy_(q_h, non_blocking=True)
-        run.segs.copy_(seg_h, non_blocking=True)
-        run.pt.copy_(pt_h, non_blocking=True)
-        tf.tf_paged_attn_decode(run.q, run.kp, run.vp, run.pt, run.segs, scale=b.scale, split_keys=b.split_keys,
-                                n_splits_max=b.n_splits_max, part_o=run.po, part_m=run.pm, part_l=run.pl,
-                                part_flag=run.pf, status=run.st, segs_host=b.segs)
+    def step(k):
+        x = run.sets[k % len(run.sets)]
+        x["q"].copy_(q_h, non_blocking=True)
+        x["segs"].copy_(seg_h, non_blocking=True)
+        x["pt"].copy_(pt_h, non_blocking=True)
+        tf.tf_paged_attn_decode(x["q"], x["kp"], x["vp"], x["pt"], x["segs"], scale=b.scale,
+                                split_keys=b.split_keys, n_splits_max=b.n_splits_max, part_o=run.po, part_m=run.pm,
+                                part_l=run.pl, part_flag=run.pf, status=run.st, segs_host=b.segs)
         tf.tf_attn_merge(run.po, run.pm, run.pl, run.pf, run.out, run.fl)
         out_h.copy_(run.out, non_blocking=True)
         fl_h.copy_(run.fl, non_blocking=True)
 
-    for _ in range(3):
-        step()
+    for k in range(3):
+        step(k)
     barrier()
-    _, total = timed_steps([step], steps, flush)
+    _, total = timed_steps([step], steps)
     barrier()
     total = max_over_ranks(total)
     ms = total / steps
@@ -401,16 +404,16 @@ def e2e_decode(b, run, flush, steps, barrier, max_over_ranks, world):
             "path": "binding tf_paged_attn_decode + tf_attn_merge, pinned host buffers"}
 
 
-def bench_verify(wl, dev, flush, steps, peaks, traffic):
+def bench_verify(wl, dev, steps, peaks, traffic):
     b = wl.shared_verify(3)
     rows = b.n_rows_total
     logits = wl.verify_logits(3, rows)
-    run = DecodeRun(b, dev, logits)
-    for _ in range(3):
-        run.partial()
-        run.merge()
-        run.argmax()
-    per, total = timed_steps([run.partial, run.merge, run.argmax], steps, flush)
+    run = DecodeRun(b, dev, logits, copies=8)  # 8 x (151 MB of KV + 17 MB of logits)
+    for k in range(3):
+        run.partial(k)
+        run.merge(k)
+        run.argmax(k)
+    per, total = timed_steps([run.partial, run.merge, run.argmax], steps)
     kv = b.kv_bytes()
     pms, mms, ams = per[0] / steps, per[1] / steps, per[2] / steps
     flops = 4 * b.head_dim * sum(int(s[1]) * b.n_q_heads * (int(s[2]) - int(s[1]) + 1) + b.n_q_heads *
@@ -423,7 +426,7 @@ def bench_verify(wl, dev, flush, steps, peaks, traffic):
                    "tflops": round(flops / (pms * 1e-3) / 1e12, 2),
                    "roofline": roofline("hbm", kv / (pms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                         traffic.get("decode_partial_cfg3")),
-                   "launches": 2 * steps},
+                   "launches": 2 * steps, "l2": "8 rotating copies"},
         "argmax": {"workload": f"{rows} rows x 128,000 bf16 ~N(0,3), ties in ~1/4 of rows",
                    "rows_per_s": round(rows / (ams * 1e-3), 1), "ms": round(ams, 5),
                    "roofline": roofline("hbm", arg_bytes / (ams * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
@@ -434,7 +437,7 @@ def bench_verify(wl, dev, flush, steps, peaks, traffic):
     return out
 
 
-def bench_ring(wl, tf, dev, flush, steps, peaks):
+def bench_ring(wl, tf, dev, steps, peaks):
     import torch
 
     from paged_kv_cache_segment_b200 import binding
@@ -442,46 +445,51 @@ def bench_ring(wl, tf, dev, flush, steps, peaks):
     b = wl.drafter_ring(5)
     n = len(b.rsegs)
     hq, d = b.n_q_heads, b.head_dim
-    q, rk, rv = to_dev(b.q, dev), to_dev(b.ring_k, dev), to_dev(b.ring_v, dev)
-    rs = binding.rsegs_to_device(b.rsegs, dev)
+    sets = [dict(q=to_dev(b.q, dev), rk=to_dev(b.ring_k, dev), rv=to_dev(b.ring_v, dev),
+                 rs=binding.rsegs_to_device(b.rsegs, dev)) for _ in range(3)]  # 3 x 146 MB of rings
     ws = torch.empty(tf.tf_ring_workspace_bytes(n, hq, d, b.n_splits_max), dtype=torch.uint8, device=dev)
     out = torch.empty((n, hq, d), device=dev)
     fl = torch.empty((n, hq), dtype=torch.uint8, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def step():
-        tf.tf_ring_attn(q, rk, rv, rs, scale=b.scale, split_slots=b.split_slots, n_splits_max=b.n_splits_max,
-                        workspace=ws, out=out, flags=fl, status=st, rsegs_host=b.rsegs)
+    def step(k):
+        x = sets[k % 3]
+        tf.tf_ring_attn(x["q"], x["rk"], x["rv"], x["rs"], scale=b.scale, split_slots=b.split_slots,
+                        n_splits_max=b.n_splits_max, workspace=ws, out=out, flags=fl, status=st, rsegs_host=b.rsegs)
 
-    for _ in range(3):
-        step()
-    per, total = timed_steps([step], steps, flush)
+    for k in range(3):
+        step(k)
+    per, total = timed_steps([step], steps)
     ms = total / steps
     kv = b.kv_bytes()
     assert int(st.item()) == 0
     return {"workload": "drafter ring: 17 rows, rings of 4,200 slots, random heads, U{1000..4200} valid, 16/2 heads, "
                         "D256, 256-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
             "ms_per_step": round(ms, 5), "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
-            "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"), "launches": 2 * steps}
+            "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"), "launches": 2 * steps,
+            "l2": "3 rotating copies"}
 
 
-def bench_prompt(wl, tf, dev, flush, steps, peaks):
+def bench_prompt(wl, tf, dev, steps, peaks):
     import torch
 
     b, spans = wl.long_prompt(4)
     rows, hq, d = b.q.shape
-    q, kp, vp, pt = to_dev(b.q, dev), to_dev(b.k_pool, dev), to_dev(b.v_pool, dev), to_dev(b.page_table, dev)
+    sets = [dict(q=to_dev(b.q, dev), kp=to_dev(b.k_pool, dev), vp=to_dev(b.v_pool, dev), pt=to_dev(b.page_table, dev))
+            for _ in range(2)]  # 2 x 184 MB
     out = torch.empty((rows, hq, d), dtype=torch.bfloat16, device=dev)
     fl = torch.empty((rows, hq), dtype=torch.uint8, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     segs = [wl.prompt_chunk_seg(b, r0, r1) for r0, r1 in spans]
 
-    def step():
+    def step(k):
+        x = sets[k % 2]
         for sg in segs:
-            tf.tf_paged_attn_prompt(q, kp, vp, pt, sg, scale=b.scale, out=out, flags=fl, status=st)
+            tf.tf_paged_attn_prompt(x["q"], x["kp"], x["vp"], x["pt"], sg, scale=b.scale, out=out, flags=fl,
+                                    status=st)
 
-    step()
-    per, total = timed_steps([step], steps, flush)
+    step(0)
+    per, total = timed_steps([step], steps)
     ms = total / steps
     n = rows
     flops = 4 * d * hq * n * (n + 1) // 2
@@ -490,7 +498,8 @@ def bench_prompt(wl, tf, dev, flush, steps, peaks):
     return {"workload": "long causal prompt: 15,000 tokens in 2,048-row chunks, 16/4 heads, D256, P32, 469 shuffled "
                         "pages, bf16 out", "tflops": round(tfl, 2), "ms_per_step": round(ms, 4),
             "algorithmic_flops": flops,
-            "roofline": roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s"), "launches": len(segs) * steps}
+            "roofline": roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s"), "launches": len(segs) * steps,
+            "l2": "2 rotating copies"}
 
 
 def cpu_baseline(b, seconds):

@@ -57,6 +57,26 @@ tf_status check_segs_host(const tf_seg *sh, int n_segs, int n_rows_total, int pa
     return TF_OK;
 }
 
+tf_status ring_merge(const float *po, const float *pm, const float *pl, const uint8_t *pf, int n_segs, int n_q_heads,
+                     int head_dim, int n_splits_max, int n_rows_total, const tf_ring_seg *rsegs, int split_slots,
+                     int64_t ring_slots_total, float *out, uint8_t *flags, cudaStream_t st) {
+    MergeParams mp{};
+    mp.part_o = po;
+    mp.part_m = pm;
+    mp.part_l = pl;
+    mp.part_flag = pf;
+    mp.n_units = (int64_t)n_segs * n_q_heads;
+    mp.n_parts = n_splits_max;
+    mp.hq = n_q_heads;
+    mp.n_rows_total = n_rows_total;
+    mp.rsegs = rsegs;
+    mp.split_slots = split_slots;
+    mp.ring_slots_total = ring_slots_total;
+    mp.out = out;
+    mp.flags = flags;
+    return cuda_status(launch_merge(mp, head_dim, true, st));
+}
+
 }  // namespace
 
 extern "C" {
@@ -91,6 +111,43 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
     }
     const int64_t n_qgroups = ((int64_t)max_rows * group + 63) / 64;
     if (n_qgroups * n_kv_heads > 65535 || n_splits_max > (1 << 30)) return TF_ERR_UNSUPPORTED;
+
+    // decode-shaped calls (a host table, at most 8 queries per stream and
+    // kv-head, splits aligned to the page boxes) take the warp-specialized kernel
+    const int tile_keys = 64;  // the warp-specialized kernel's tile
+    const int box_rows = page_size < tile_keys ? page_size : tile_keys;
+    if (segs_host && (int64_t)max_rows * group <= 8 && decode_ws_supported(head_dim, n_segs) &&
+        (split_keys == 0 || split_keys % box_rows == 0)) {
+        int64_t items = 0;
+        for (int s = 0; s < n_segs; ++s) {
+            const tf_seg e = segs_host[s];
+            if (e.n_rows == 0) continue;
+            const int per = split_len(e.n_keys, split_keys, n_splits_max, page_size);
+            items += (int64_t)((e.n_keys + per - 1) / per) * n_kv_heads;
+        }
+        WsParams w{};
+        w.q = static_cast<const uint16_t *>(q);
+        w.n_rows_total = n_rows_total;
+        w.hq = n_q_heads;
+        w.hkv = n_kv_heads;
+        w.group = group;
+        w.n_segs = n_segs;
+        w.segs = segs;
+        w.page_table = page_table;
+        w.n_pages = n_pages;
+        w.log2_page = lp;
+        w.pt_len = page_table_len;
+        w.scale_log2 = scale * 1.4426950408889634f;
+        w.split_keys = split_keys;
+        w.n_splits_max = n_splits_max;
+        w.part_o = part_o;
+        w.part_m = part_m;
+        w.part_l = part_l;
+        w.part_flag = part_flag;
+        w.status = status;
+        return cuda_status(
+            launch_decode_ws(w, head_dim, false, k_pool, v_pool, items, reinterpret_cast<cudaStream_t>(stream)));
+    }
 
     AttnParams p{};
     p.q = static_cast<const uint16_t *>(q);
@@ -250,6 +307,32 @@ tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, c
     float *pm = po + parts * head_dim;
     float *pl = pm + parts;
     uint8_t *pf = reinterpret_cast<uint8_t *>(pl + parts);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    cudaError_t e = cudaSuccess;
+    if (group <= 8 && decode_ws_supported(head_dim, n_segs) && ring_slots_total <= 0x7fffffff) {
+        WsParams w{};
+        w.q = static_cast<const uint16_t *>(q);
+        w.n_rows_total = n_rows_total;
+        w.hq = n_q_heads;
+        w.hkv = n_kv_heads;
+        w.group = group;
+        w.n_segs = n_segs;
+        w.rsegs = rsegs;
+        w.ring_slots_total = ring_slots_total;
+        w.scale_log2 = scale * 1.4426950408889634f;
+        w.split_keys = split_slots;
+        w.n_splits_max = n_splits_max;
+        w.part_o = po;
+        w.part_m = pm;
+        w.part_l = pl;
+        w.part_flag = pf;
+        w.status = status;
+        e = launch_decode_ws(w, head_dim, true, ring_k, ring_v, (int64_t)n_segs * n_kv_heads * n_splits_max, st);
+        if (e != cudaSuccess) return TF_ERR_CUDA;
+        return ring_merge(po, pm, pl, pf, n_segs, n_q_heads, head_dim, n_splits_max, n_rows_total, rsegs, split_slots,
+                          ring_slots_total, out, flags, st);
+    }
 
     AttnParams p{};
     p.q = static_cast<const uint16_t *>(q);
@@ -270,25 +353,11 @@ tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, c
     p.part_l = pl;
     p.part_flag = pf;
     p.status = status;
-    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const dim3 grid((unsigned)n_splits_max, (unsigned)(n_qgroups * n_kv_heads), (unsigned)n_segs);
-    cudaError_t e = launch_attn_partial(p, head_dim, true, false, grid, st);
+    e = launch_attn_partial(p, head_dim, true, false, grid, st);
     if (e != cudaSuccess) return TF_ERR_CUDA;
-    MergeParams mp{};
-    mp.part_o = po;
-    mp.part_m = pm;
-    mp.part_l = pl;
-    mp.part_flag = pf;
-    mp.n_units = (int64_t)n_segs * n_q_heads;
-    mp.n_parts = n_splits_max;
-    mp.hq = n_q_heads;
-    mp.n_rows_total = n_rows_total;
-    mp.rsegs = rsegs;
-    mp.split_slots = split_slots;
-    mp.ring_slots_total = ring_slots_total;
-    mp.out = out;
-    mp.flags = flags;
-    return cuda_status(launch_merge(mp, head_dim, true, st));
+    return ring_merge(po, pm, pl, pf, n_segs, n_q_heads, head_dim, n_splits_max, n_rows_total, rsegs, split_slots,
+                      ring_slots_total, out, flags, st);
 }
 
 tf_status tf_argmax_rows(const void *logits, int32_t n_rows, int32_t n_cols, int64_t ld, int32_t *ids,

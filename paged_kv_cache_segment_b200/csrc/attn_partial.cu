@@ -564,10 +564,15 @@ __global__ void __launch_bounds__(kThreads, (D == 256) ? 1 : 2) attn_partial_ker
 // ---------------------------------------------------------------------------
 // merge: one warp per (row, q-head) unit
 // ---------------------------------------------------------------------------
+// Lane c holds partial c's weight e^(m_c - M) (0 for an empty partial); the o
+// rows are then read with independent, predicated loads four partials at a
+// time.  The kernel may be launched as a programmatic dependent of the
+// partial kernel: it waits for that grid before reading.
 template <int D, bool RING>
-__global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t u = (int64_t)blockIdx.x * 8 + warp;
+    const int64_t u = (int64_t)blockIdx.x * 4 + warp;
     if (u >= p.n_units) return;
     int64_t out_u = u;
     int C = p.n_parts;
@@ -593,52 +598,81 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
     const float *pm = p.part_m + u * p.n_parts;
     const float *pl = p.part_l + u * p.n_parts;
     const uint8_t *pf = p.part_flag + u * p.n_parts;
-    float M = -INFINITY;
+    const float *po = p.part_o + u * p.n_parts * D;
+
+    // Everything a chunk of up to 16 partials needs is loaded in one round:
+    // lane c's (m, l, flag) and every lane's slice of each o row.  An empty
+    // partial's o is never multiplied in (its weight selects 0), so its
+    // unwritten contents cannot leak into the sum.
+    constexpr int NV = (D + 127) / 128;
+    constexpr int CH = 16;
+    float4 acc[NV];
+#pragma unroll
+    for (int k = 0; k < NV; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float M = -INFINITY, L = 0.f;
     uint32_t f = 0, any = 0;
-    for (int c = lane; c < C; c += 32) {
-        const float lc = pl[c];
-        f |= pf[c];
-        if (lc > 0.f) {
-            any = 1;
-            M = fmaxf(M, pm[c]);
+    for (int c0 = 0; c0 < C; c0 += CH) {
+        const int n = min(CH, C - c0);
+        float4 v[CH][NV];
+#pragma unroll
+        for (int j = 0; j < CH; ++j)
+#pragma unroll
+            for (int k = 0; k < NV; ++k) {
+                const int d0 = k * 128 + lane * 4;
+                v[j][k] = (j < n && d0 < D) ? *reinterpret_cast<const float4 *>(po + (int64_t)(c0 + j) * D + d0)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        float mc = -INFINITY, lc = 0.f;
+        if (lane < n) {
+            mc = pm[c0 + lane];
+            lc = pl[c0 + lane];
+            f |= pf[c0 + lane];
         }
-    }
+        const bool live = lc > 0.f;
+        if (live) any = 1;
+        // chunk max, merged into the running max (rescaling what came before)
+        float mx = live ? mc : -INFINITY;
 #pragma unroll
-    for (int x = 16; x; x >>= 1) {
-        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
-        f |= __shfl_xor_sync(0xffffffffu, f, x);
-        any |= __shfl_xor_sync(0xffffffffu, any, x);
-    }
-    float L = 0.f;
-    for (int c = lane; c < C; c += 32) {
-        const float lc = pl[c];
-        if (lc > 0.f) L += ex2((pm[c] - M) * kLog2e) * lc;
-    }
+        for (int x = 16; x; x >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+        const float Mn = fmaxf(M, mx);
+        if (Mn != -INFINITY) {
+            const float r = (M == -INFINITY) ? 0.f : ex2((M - Mn) * kLog2e);
+            L *= r;
 #pragma unroll
-    for (int x = 16; x; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
-    bool nf = !isfinite(L) || !any;
-    float4 acc[(D + 127) / 128];
+            for (int k = 0; k < NV; ++k) {
+                acc[k].x *= r;
+                acc[k].y *= r;
+                acc[k].z *= r;
+                acc[k].w *= r;
+            }
+            M = Mn;
+        }
+        const float w = live ? ex2((mc - M) * kLog2e) : 0.f;
+        L += w * lc;  // lane-partial, reduced below
 #pragma unroll
-    for (int k = 0; k < (D + 127) / 128; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < C; ++c) {
-        const float lc = pl[c];
-        if (!(lc > 0.f)) continue;
-        const float wc = ex2((pm[c] - M) * kLog2e);
-        const float *oc = p.part_o + (u * p.n_parts + c) * D;
+        for (int j = 0; j < CH; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, w, j);
+            if (j < n && wj != 0.f) {
 #pragma unroll
-        for (int k = 0; k < (D + 127) / 128; ++k) {
-            const int d0 = k * 128 + lane * 4;
-            if (d0 < D) {
-                const float4 v = *reinterpret_cast<const float4 *>(oc + d0);
-                acc[k].x += wc * v.x;
-                acc[k].y += wc * v.y;
-                acc[k].z += wc * v.z;
-                acc[k].w += wc * v.w;
+                for (int k = 0; k < NV; ++k) {
+                    acc[k].x += wj * v[j][k].x;
+                    acc[k].y += wj * v[j][k].y;
+                    acc[k].z += wj * v[j][k].z;
+                    acc[k].w += wj * v[j][k].w;
+                }
             }
         }
     }
 #pragma unroll
-    for (int k = 0; k < (D + 127) / 128; ++k) {
+    for (int x = 16; x; x >>= 1) {
+        f |= __shfl_xor_sync(0xffffffffu, f, x);
+        any |= __shfl_xor_sync(0xffffffffu, any, x);
+    }
+#pragma unroll
+    for (int x = 16; x; x >>= 1) L += __shfl_xor_sync(0xffffffffu, L, x);
+    bool nf = !isfinite(L) || !any;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
         const int d0 = k * 128 + lane * 4;
         if (d0 < D) {
             acc[k].x /= L;
@@ -650,7 +684,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
     }
     f |= __any_sync(0xffffffffu, nf) ? 1u : 0u;
 #pragma unroll
-    for (int k = 0; k < (D + 127) / 128; ++k) {
+    for (int k = 0; k < NV; ++k) {
         const int d0 = k * 128 + lane * 4;
         if (d0 < D) {
             const float4 v = f ? make_float4(qnan, qnan, qnan, qnan) : acc[k];
@@ -690,23 +724,31 @@ cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bo
     return launch_partial_d<Src::kPaged, false>(p, head_dim, grid, st);
 }
 
+template <int D, bool RING>
+static cudaError_t launch_merge_t(const MergeParams &p, cudaStream_t st) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((p.n_units + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, merge_kernel<D, RING>, p);
+}
+
 cudaError_t launch_merge(const MergeParams &p, int head_dim, bool ring, cudaStream_t st) {
     if (p.n_units == 0) return cudaSuccess;
-    const dim3 grid((unsigned)((p.n_units + 7) / 8));
-#define TF_MERGE_CASE(DV)                                              \
-    case DV:                                                           \
-        if (ring)                                                      \
-            merge_kernel<DV, true><<<grid, 256, 0, st>>>(p);           \
-        else                                                           \
-            merge_kernel<DV, false><<<grid, 256, 0, st>>>(p);          \
-        break;
+    cudaError_t e;
     switch (head_dim) {
-        TF_MERGE_CASE(64)
-        TF_MERGE_CASE(128)
-        TF_MERGE_CASE(256)
+        case 64: e = ring ? launch_merge_t<64, true>(p, st) : launch_merge_t<64, false>(p, st); break;
+        case 128: e = ring ? launch_merge_t<128, true>(p, st) : launch_merge_t<128, false>(p, st); break;
+        case 256: e = ring ? launch_merge_t<256, true>(p, st) : launch_merge_t<256, false>(p, st); break;
         default: return cudaErrorInvalidValue;
     }
-#undef TF_MERGE_CASE
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -31,6 +31,7 @@
 #include "tf_common.cuh"
 #include "tf_internal.h"
 #include "tf_sm100.cuh"
+#include "tma_host.h"
 
 namespace tfp {
 
@@ -302,10 +303,10 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         // tensor memory is released
         if (tid == 0) report_timeout(p.status);
         for (int i = 0; i < 2; ++i) {
-            mbar_wait(bk, (uint32_t)i, 1u << 12);
-            mbar_wait(bv, (uint32_t)i, 1u << 12);
-            mbar_wait(bs, (uint32_t)i, 1u << 12);
-            mbar_wait(bo, (uint32_t)i, 1u << 12);
+            mbar_wait(bk, (uint32_t)i, 20000000ull);
+            mbar_wait(bv, (uint32_t)i, 20000000ull);
+            mbar_wait(bs, (uint32_t)i, 20000000ull);
+            mbar_wait(bo, (uint32_t)i, 20000000ull);
         }
     }
     uint32_t bad = (emax == 0x7f800000u) | tail_bad | (uint32_t)s_err | timed_out;
@@ -367,32 +368,6 @@ __global__ void __launch_bounds__(kPTThreads, 1)
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-static bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
-                     const cuuint32_t *box) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 bool prompt_tc_supported(int head_dim, int group, int page_size) {
     return (head_dim == 64 || head_dim == 128 || head_dim == 256) && group >= 1 && group <= 128 &&
            (128 % group) == 0 && page_size >= 8;
@@ -407,14 +382,14 @@ static cudaError_t launch_prompt_tc_t(const PromptTcParams &p, const void *q, co
         const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.hq, (cuuint64_t)p.n_rows_total};
         const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.hq * D * 2};
         const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)RT};
-        if (!make_map(&mq, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tensor_map_bf16(&mq, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
     }
     {
         const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)p.hkv, (cuuint64_t)p.n_pages};
         const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)P * D * 2, (cuuint64_t)p.hkv * P * D * 2};
         const cuuint32_t box[4] = {64, (cuuint32_t)BR, 1, 1};
-        if (!make_map(&mk, k, 4, dims, strides, box)) return cudaErrorInvalidValue;
-        if (!make_map(&mv, v, 4, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tensor_map_bf16(&mk, k, 4, dims, strides, box)) return cudaErrorInvalidValue;
+        if (!make_tensor_map_bf16(&mv, v, 4, dims, strides, box)) return cudaErrorInvalidValue;
     }
     auto kern = prompt_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PTCfg<D>::kSmemBytes);

@@ -59,6 +59,25 @@ struct PromptTcParams {
     uint32_t *status;
 };
 
+// Parameters of the warp-specialized decode kernel (paged or ring source).
+struct WsParams {
+    const uint16_t *q;
+    int n_rows_total, hq, hkv, group;
+    int n_segs;
+    // paged
+    const tf_seg *segs;
+    const int32_t *page_table;
+    int n_pages, log2_page, pt_len;
+    // ring
+    const tf_ring_seg *rsegs;
+    int64_t ring_slots_total;
+    float scale_log2;
+    int split_keys, n_splits_max;
+    float *part_o, *part_m, *part_l;
+    uint8_t *part_flag;
+    uint32_t *status;
+};
+
 struct ArgmaxParams {
     const uint16_t *logits;
     int n_rows, n_cols;
@@ -72,6 +91,9 @@ cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bo
 cudaError_t launch_merge(const MergeParams &p, int head_dim, bool ring, cudaStream_t st);
 cudaError_t launch_argmax(const ArgmaxParams &p, bool vec, cudaStream_t st);
 bool prompt_tc_supported(int head_dim, int group, int page_size);
+bool decode_ws_supported(int head_dim, int n_segs);
+cudaError_t launch_decode_ws(const WsParams &p, int head_dim, bool ring, const void *k, const void *v,
+                             int64_t n_items_bound, cudaStream_t st);
 cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *q, const void *k, const void *v,
                              cudaStream_t st);
 

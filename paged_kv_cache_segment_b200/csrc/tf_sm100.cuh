@@ -24,6 +24,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
     uint32_t ok;
     asm volatile(
@@ -36,13 +40,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
     return ok != 0;
 }
 
-// Wait for phase `phase` of a barrier, giving up after `limit` polls (each
-// poll may suspend the thread for a hardware-defined while).  Returns false on
-// timeout so the caller can report it instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, uint32_t limit = (1u << 24)) {
-    for (uint32_t i = 0; i < limit; ++i)
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `phase` of a barrier, giving up after `limit_ns` nanoseconds
+// of the global timer (2 s by default: every legitimate wait here is a few
+// microseconds).  Returns false on timeout so the caller can report it instead
+// of hanging.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, uint64_t limit_ns = 2000000000ull) {
+    for (int i = 0; i < 64; ++i)
         if (mbar_try_wait(bar, phase)) return true;
-    return false;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, phase)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // Generic-proxy writes to shared memory become visible to the async proxy.
@@ -69,8 +84,41 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// Untiled bulk copy global -> shared (both 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one row pair per thread.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Barrier among `count` threads on hardware barrier `id` (id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier among `count` threads that also ORs a predicate over them.
+__device__ __forceinline__ bool named_bar_red_or(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %3, 0;\n\t"
+        "bar.red.or.pred po, %1, %2, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"(id), "r"(count), "r"(pred ? 1u : 0u)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------- tensor memory

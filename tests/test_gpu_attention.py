@@ -311,9 +311,11 @@ def test_ring_wrap_cases(orc, size, head, n):
 
 def test_ring_equals_unrolled_paged_byte_for_byte():
     """A ring read oldest-first equals the same keys laid out contiguously
-    and read by the paged kernel, bit for bit (same tiles, same fold order)."""
-    b = wl.make_ring_batch(80, n_streams=2, ring_size=700, valid_lo=650, valid_hi=690, n_q_heads=16, n_kv_heads=2,
-                           head_dim=256, split_slots=128)
+    and read by the paged kernel, bit for bit, when the wrap falls on a tile
+    boundary (same tiles, same fold order)."""
+    # ring 0 does not wrap; ring 1 wraps at key 128, on a 64-key tile boundary
+    b = wl.make_ring_batch(80, n_streams=2, ring_size=700, valid_lo=640, valid_hi=640, n_q_heads=16, n_kv_heads=2,
+                           head_dim=256, split_slots=128, heads=[640, 512], valids=[640, 640])
     r = run_ring(b)
     for s in range(2):
         e = b.rsegs[s]
