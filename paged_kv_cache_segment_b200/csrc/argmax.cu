@@ -6,15 +6,19 @@
 // flagged.  Readings: values compare as real numbers (-0 == +0), a flagged
 // row reports id -1.
 //
-// Each row is split over a cluster of 8 CTAs.  Every CTA streams its share of
-// the row with 16-byte loads, keeps per thread the first column holding its
-// largest value, reduces over its warps, and the cluster's rank-0 CTA folds
-// the 8 CTA results through distributed shared memory.  No workspace and no
-// inter-CTA counters: the cluster barrier orders the exchange.
-//
-// Comparing bf16 values as reals uses an order-preserving 16-bit key: for a
-// non-negative value the bits with the sign bit set, for a negative value all
-// bits inverted, and -0 mapped to +0 first.
+// Each row is split over a cluster of 8 CTAs.  Every thread loads its share
+// with 16-byte loads (eight in flight) and works on 32-bit words, two bf16
+// values each: max.bf16x2 keeps the largest value of each half and
+// max.u16x2 over the magnitude bits keeps the largest exponent pattern
+// (reaching 0x7f80 means a NaN or an infinity).  The cluster agrees on the
+// row's largest value (each CTA stores its block maximum, as an
+// order-preserving 16-bit key, into every CTA's shared memory; one cluster
+// barrier; local reads), then each thread finds the first column equal to it
+// among the words it still holds in registers (an IEEE compare, so -0 equals
+// +0), and the CTAs' first columns meet on rank 0 the same way.  No
+// workspace and no inter-CTA counters: the cluster barriers order the
+// exchanges.
+
 #include <cooperative_groups.h>
 
 #include <climits>
@@ -29,115 +33,145 @@ namespace tfp {
 
 constexpr int kArgThreads = 256;
 constexpr int kArgBatch = 8;  // 16-byte vectors in flight per thread
+constexpr int kArgWarps = kArgThreads / 32;
 
-__device__ __forceinline__ uint32_t order_key(uint32_t b) {
-    b = (b == 0x8000u) ? 0u : b;
-    return (b & 0x8000u) ? (b ^ 0xffffu) : (b | 0x8000u);
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
-
-__device__ __forceinline__ void take(uint32_t b, int col, uint32_t &best, int &best_col, uint32_t &bad) {
-    bad |= ((b & 0x7f80u) == 0x7f80u);
-    const uint32_t k = order_key(b);
-    if (k > best) {
-        best = k;
-        best_col = col;
-    }
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
-
-// (key, col) pairs: the larger key wins, then the lower column.
-__device__ __forceinline__ void better_of(uint32_t &k, int &c, uint32_t k2, int c2) {
-    if (k2 > k || (k2 == k && c2 < c)) {
-        k = k2;
-        c = c2;
-    }
+// Per half: 0xffff where the two bf16 values are equal (so -0 equals +0).
+__device__ __forceinline__ uint32_t eq_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("set.eq.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
+// Order-preserving 16-bit key of one bf16 value, and back.
+__device__ __forceinline__ uint32_t key16(uint32_t b) { return (b & 0x8000u) ? (b ^ 0xffffu) : (b | 0x8000u); }
+__device__ __forceinline__ uint32_t unkey16(uint32_t k) { return (k & 0x8000u) ? (k ^ 0x8000u) : (k ^ 0xffffu); }
 
 template <bool VEC>
 __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThreads) argmax_kernel(const ArgmaxParams p) {
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ uint32_t w_key[kArgThreads / 32], w_bad[kArgThreads / 32];
-    __shared__ int w_col[kArgThreads / 32];
-    __shared__ uint32_t c_key, c_bad;
-    __shared__ int c_col;
+    __shared__ uint32_t w_red[kArgWarps];
+    __shared__ uint32_t x_max[kArgmaxCluster];  // filled by every CTA of the cluster
+    __shared__ int x_idx[kArgmaxCluster];       // filled on rank 0
 
     // columns per CTA, a multiple of 8 so vectors never straddle two CTAs
     const int per = ((p.n_cols + kArgmaxCluster * 8 - 1) / (kArgmaxCluster * 8)) * 8;
     const int c0 = min(p.n_cols, rank * per), c1 = min(p.n_cols, c0 + per);
+    const uint32_t kNegInf2 = 0xff80ff80u, kPad2 = 0xff7fff7fu;
 
     for (int row = blockIdx.y; row < p.n_rows; row += gridDim.y) {
         const uint16_t *rp = p.logits + (int64_t)row * p.ld;
-        uint32_t best = 0u, bad = 0u;
-        int best_col = INT_MAX;
+        // ---- pass 1: the largest value and the largest magnitude pattern
+        uint32_t words[kArgBatch * 4];
+        uint32_t vmax = kNegInf2, mag = 0u;
+        const uint4 *vp = reinterpret_cast<const uint4 *>(rp);
+        const int v0 = c0 >> 3, v1 = VEC ? (c1 >> 3) : v0;
         if constexpr (VEC) {
-            const uint4 *vp = reinterpret_cast<const uint4 *>(rp);
-            const int v0 = c0 >> 3, v1 = c1 >> 3;  // whole vectors [v0, v1)
-            for (int vb = v0 + tid; vb < v1; vb += kArgThreads * kArgBatch) {
-                uint4 buf[kArgBatch];
+            // a thread's vectors are v0 + tid + k * kArgThreads
 #pragma unroll
-                for (int k = 0; k < kArgBatch; ++k) {
-                    const int v = vb + k * kArgThreads;
-                    buf[k] = v < v1 ? __ldg(vp + v) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
-                }
+            for (int k = 0; k < kArgBatch; ++k) {
+                const int v = v0 + tid + k * kArgThreads;
+                // padding: the most negative finite bf16 (leaves the max and the
+                // magnitude test alone; pass 2 skips it by its vector index)
+                const uint4 x = v < v1 ? __ldg(vp + v) : make_uint4(kPad2, kPad2, kPad2, kPad2);
+                words[4 * k] = x.x;
+                words[4 * k + 1] = x.y;
+                words[4 * k + 2] = x.z;
+                words[4 * k + 3] = x.w;
+            }
 #pragma unroll
-                for (int k = 0; k < kArgBatch; ++k) {
-                    const int v = vb + k * kArgThreads;
-                    if (v < v1) {
-                        const uint32_t wd[4] = {buf[k].x, buf[k].y, buf[k].z, buf[k].w};
+            for (int k = 0; k < kArgBatch * 4; ++k) {
+                vmax = max_bf16x2(vmax, words[k]);
+                mag = max_u16x2(mag, words[k] & 0x7fff7fffu);
+            }
+            // vectors past the ones held (rows wider than 8 x 256 x 8 columns a CTA)
+            for (int v = v0 + tid + kArgBatch * kArgThreads; v < v1; v += kArgThreads) {
+                const uint4 x = __ldg(vp + v);
+                const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            take(wd[e] & 0xffffu, v * 8 + 2 * e, best, best_col, bad);
-                            take(wd[e] >> 16, v * 8 + 2 * e + 1, best, best_col, bad);
-                        }
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    vmax = max_bf16x2(vmax, wd[e]);
+                    mag = max_u16x2(mag, wd[e] & 0x7fff7fffu);
                 }
             }
-            // ragged tail of the row (last CTA only)
-            for (int c = (v1 << 3) + tid; c < c1; c += kArgThreads) take(rp[c], c, best, best_col, bad);
-        } else {
-            for (int c = c0 + tid; c < c1; c += kArgThreads) take(rp[c], c, best, best_col, bad);
         }
-        // warp, then CTA
+        // scalar columns: the row's ragged tail, or everything without 16-byte access
+        for (int c = (VEC ? (v1 << 3) : c0) + tid; c < c1; c += kArgThreads) {
+            const uint32_t b = rp[c];
+            vmax = max_bf16x2(vmax, b | 0xff800000u);
+            mag = max_u16x2(mag, b & 0x7fffu);
+        }
+        // nonfinite: some half's magnitude pattern reached the all-ones exponent
+        const uint32_t bad = ((mag & 0xffffu) >= 0x7f80u || (mag >> 16) >= 0x7f80u) ? 1u : 0u;
+        uint32_t k = max(key16(vmax & 0xffffu), key16(vmax >> 16));
+        // ---- the cluster's largest value (as a key) and any nonfinite value
+        k = __reduce_max_sync(0xffffffffu, k);
+        const uint32_t wbad = __reduce_or_sync(0xffffffffu, bad);
+        if (lane == 0) w_red[warp] = k | (wbad << 31);
+        __syncthreads();
+        if (tid < kArgmaxCluster) {
+            uint32_t m = 0;
 #pragma unroll
-        for (int x = 16; x; x >>= 1) {
-            const uint32_t k2 = __shfl_xor_sync(0xffffffffu, best, x);
-            const int c2 = __shfl_xor_sync(0xffffffffu, best_col, x);
-            better_of(best, best_col, k2, c2);
-            bad |= __shfl_xor_sync(0xffffffffu, bad, x);
+            for (int i = 0; i < kArgWarps; ++i) m = max(m, w_red[i]);  // the flag bit rides on top
+            *cluster.map_shared_rank(&x_max[rank], tid) = m;         // every CTA tells every CTA
         }
-        if (lane == 0) {
-            w_key[warp] = best;
-            w_col[warp] = best_col;
-            w_bad[warp] = bad;
+        cluster.sync();
+        uint32_t K = 0, B = 0;
+#pragma unroll
+        for (int i = 0; i < kArgmaxCluster; ++i) {
+            K = max(K, x_max[i] & 0xffffu);
+            B |= x_max[i] >> 31;
         }
+        const uint32_t M = unkey16(K);
+        const uint32_t M2 = M | (M << 16);
+        // ---- pass 2: the first column holding the largest value
+        int best = INT_MAX;
+        if constexpr (VEC) {
+#pragma unroll
+            for (int j = 0; j < kArgBatch * 4; ++j) {
+                const uint32_t e = eq_bf16x2(words[j], M2);
+                const int v = v0 + tid + (j >> 2) * kArgThreads;
+                if (best == INT_MAX && e && v < v1) best = v * 8 + (j & 3) * 2 + ((e & 0xffffu) ? 0 : 1);
+            }
+            for (int v = v0 + tid + kArgBatch * kArgThreads; v < v1 && best == INT_MAX; v += kArgThreads) {
+                const uint4 x = __ldg(vp + v);
+                const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t e = eq_bf16x2(wd[q], M2);
+                    if (best == INT_MAX && e) best = v * 8 + 2 * q + ((e & 0xffffu) ? 0 : 1);
+                }
+            }
+        }
+        for (int c = (VEC ? (v1 << 3) : c0) + tid; c < c1 && best == INT_MAX; c += kArgThreads)
+            if (eq_bf16x2(rp[c], M) & 0xffffu) best = c;
+        best = __reduce_min_sync(0xffffffffu, best);
+        if (lane == 0) w_red[warp] = (uint32_t)best;
         __syncthreads();
         if (tid == 0) {
-            uint32_t k = w_key[0], b = w_bad[0];
-            int c = w_col[0];
-            for (int i = 1; i < kArgThreads / 32; ++i) {
-                better_of(k, c, w_key[i], w_col[i]);
-                b |= w_bad[i];
-            }
-            c_key = k;
-            c_col = c;
-            c_bad = b;
+            int b = INT_MAX;
+#pragma unroll
+            for (int i = 0; i < kArgWarps; ++i) b = min(b, (int)w_red[i]);
+            *cluster.map_shared_rank(&x_idx[rank], 0) = b;
         }
         cluster.sync();
         if (rank == 0 && tid == 0) {
-            uint32_t k = c_key, b = c_bad;
-            int c = c_col;
-            for (int r = 1; r < kArgmaxCluster; ++r) {
-                const uint32_t *rk = cluster.map_shared_rank(&c_key, r);
-                const int *rc = cluster.map_shared_rank(&c_col, r);
-                const uint32_t *rb = cluster.map_shared_rank(&c_bad, r);
-                better_of(k, c, *rk, *rc);
-                b |= *rb;
-            }
-            p.ids[row] = b ? -1 : c;
-            p.flags[row] = (uint8_t)(b ? 1 : 0);
+            int b = INT_MAX;
+#pragma unroll
+            for (int i = 0; i < kArgmaxCluster; ++i) b = min(b, x_idx[i]);
+            p.ids[row] = B ? -1 : b;
+            p.flags[row] = (uint8_t)(B ? 1 : 0);
         }
-        cluster.sync();  // rank 0 has read every CTA's result before anyone reuses it
     }
 }
 

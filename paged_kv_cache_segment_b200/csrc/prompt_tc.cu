@@ -17,9 +17,11 @@
 //   3. every thread owns one query row: it loads its S row from tensor memory,
 //      masks it causally, and folds it into a running max / sum with a lazy
 //      rescale (the reference max moves only when it rises by more than 2^8);
-//   4. the weights go back to tensor memory as bf16 hi + bf16 lo and one
-//      thread issues O += P_hi V + P_lo V (A from tensor memory, B = V in
-//      shared memory, MN-major), so each weight keeps about 16 bits;
+//   4. the weights go back to tensor memory (into the S columns they came
+//      from) and one thread issues O += P V (A from tensor memory, B = V in
+//      shared memory, MN-major).  For f32 output P is fed as bf16 hi + bf16 lo
+//      (two MMAs, about 16 bits a weight, so the fp32 tolerance holds); for
+//      bf16 output P is one bf16, whose rounding is below the output's own;
 //   5. O stays in tensor memory until the epilogue divides by the sum.
 // Nonfinite handling matches the other attention kernels: visible scores are
 // checked through their exponent bits, value rows that only some rows see
@@ -35,40 +37,64 @@
 
 namespace tfp {
 
-constexpr int kPTThreads = 128;
-constexpr int kBN = 128;                // keys per tile
-constexpr int kSlabBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16 columns)
-constexpr uint32_t kColS = 0, kColPhi = 128, kColPlo = 192, kColO = 256;
+constexpr int kPTSoftmax = 128;               // four softmax warps, one query row a thread
+constexpr int kPTThreads = kPTSoftmax + 32;   // + one issuer warp (MMAs and TMA)
+constexpr int kQM = 128;                      // queries a CTA (the MMA's M)
+constexpr int kBN = 64;                       // keys a tile
+constexpr int kQSlab = kQM * 128;             // 128 query rows x 128 bytes
+constexpr int kKVSlab = kBN * 128;            // 64 key rows x 128 bytes
+constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 256;  // tensor-memory columns
 
 template <int D>
 struct PTCfg {
     static constexpr int kSlabs = D / 64;
-    static constexpr int kTileBytes = kSlabs * kSlabBytes;  // 128 rows x D bf16
-    static constexpr int kSmemBytes = 3 * kTileBytes + 1024; // Q, K, V + alignment slack
-    static constexpr uint32_t kTmemCols = (256 + D) <= 512 ? 512 : 0;
+    static constexpr int kQBytes = kSlabs * kQSlab;
+    static constexpr int kKVBytes = kSlabs * kKVSlab;
+    // Q, two K buffers, two V buffers
+    static constexpr int kOffK = kQBytes;
+    static constexpr int kOffV = kQBytes + 2 * kKVBytes;
+    static constexpr int kPidCap = 4096;  // page ids held in shared memory (16 KB)
+    static constexpr int kOffPid = kQBytes + 4 * kKVBytes;
+    static constexpr int kSmemBytes = kOffPid + kPidCap * 4 + 1024;
+    static constexpr uint32_t kTmemCols = 512;
 };
 
-__device__ __forceinline__ void report_timeout(uint32_t *status) { atomicOr(status, TF_DEV_TIMEOUT); }
+// Bounded wait that gives up at once after any thread of the CTA gave up, so
+// every role keeps its barrier sequence without waiting twice the timeout.
+__device__ __forceinline__ bool pt_wait(uint32_t bar, uint32_t phase, volatile uint32_t *abort_flag) {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, phase)) return true;
+    *abort_flag = 1;
+    return false;
+}
 
-template <int D>
+template <int D, bool HILO>
 __global__ void __launch_bounds__(kPTThreads, 1)
     prompt_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const PromptTcParams p) {
     using C = PTCfg<D>;
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t bars[5];  // q, k, v, s, o
+    // barriers: q; k[2]; v[2]; s[2] (QK done); pr[2] (P written, V cleaned); o[2] (PV done)
+    __shared__ __align__(8) uint64_t bars[11];
     __shared__ uint32_t s_tmem;
     __shared__ uint32_t s_vbad[4];
-    __shared__ int s_err;
+    __shared__ uint32_t s_err, s_abort;
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *sbase_ptr = smem_raw + (sbase - smem_u32(smem_raw));
-    const uint32_t sQ = sbase, sK = sbase + C::kTileBytes, sV = sbase + 2 * C::kTileBytes;
-    const uint32_t bq = smem_u32(&bars[0]), bk = smem_u32(&bars[1]), bv = smem_u32(&bars[2]),
-                   bs = smem_u32(&bars[3]), bo = smem_u32(&bars[4]);
+    const uint32_t sQ = sbase;
+    auto sK = [&](int b) { return sbase + C::kOffK + b * C::kKVBytes; };
+    auto sV = [&](int b) { return sbase + C::kOffV + b * C::kKVBytes; };
+    const uint32_t bq = smem_u32(&bars[0]);
+    auto bk = [&](int b) { return smem_u32(&bars[1 + b]); };
+    auto bv = [&](int b) { return smem_u32(&bars[3 + b]); };
+    auto bsq = [&](int b) { return smem_u32(&bars[5 + b]); };
+    auto bpr = [&](int b) { return smem_u32(&bars[7 + b]); };
+    auto bo = [&](int b) { return smem_u32(&bars[9 + b]); };
+    volatile uint32_t *abort_flag = &s_abort;
 
-    const int G = p.group, RT = kBN / p.group;  // rows per tile
+    const int G = p.group, RT = kQM / p.group;  // rows a tile
     const int g = blockIdx.y;
     const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;  // the most keys first
     const int row0 = qt * RT;                              // chunk-relative first row
@@ -79,240 +105,284 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     const int n_tiles = (key_hi_eff + kBN - 1) / kBN;
     const int P = 1 << p.log2_page, BR = P < kBN ? P : kBN, n_box = kBN / BR;
 
+    // The CTA's page ids, read once here by every thread (coalesced), so the
+    // issuer never waits on a page-table read inside the key loop.
+    int *pids = reinterpret_cast<int *>(sbase_ptr + C::kOffPid);
+    const int n_pid = min((key_hi_eff + P - 1) >> p.log2_page, p.n_pg);
+    for (int i = tid; i < n_pid && i < C::kPidCap; i += kPTThreads) {
+        const int id = p.page_table[p.pt_base + i];
+        pids[i] = (id < 0 || id >= p.n_pages) ? -1 : id;
+    }
     if (warp == 0) {
         tmem_alloc(smem_u32(&s_tmem), C::kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(smem_u32(&bars[i]), 1);
+        for (int i = 0; i < 11; ++i) mbar_init(smem_u32(&bars[i]), (i >= 7 && i <= 8) ? 4u : 1u);
         fence_barrier_init();
         s_err = 0;
+        s_abort = 0;
         s_vbad[0] = s_vbad[1] = s_vbad[2] = s_vbad[3] = 0;
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 
-    // K or V tile t into its buffer: one box per page (or per 128-key span of a
-    // larger page); page ids are read once here, the tile's only lookup.
-    auto issue_kv = [&](int t, bool is_v) {
-        const int kt = t * kBN;
-        const uint32_t dst0 = is_v ? sV : sK;
-        const uint32_t bar = is_v ? bv : bk;
-        const CUtensorMap *map = is_v ? &tmV : &tmK;
-        int pid[16];
-        uint32_t bytes = 0;
-        for (int b = 0; b < n_box; ++b) {
-            const int key0 = kt + b * BR;
-            int id = -1;
-            if (key0 < key_hi_eff) {
-                const int idx = key0 >> p.log2_page;
-                id = (idx < p.n_pg) ? p.page_table[p.pt_base + idx] : -2;
-                if (id < 0 || id >= p.n_pages) {
-                    id = -1;
-                    s_err = 1;
-                    atomicOr(p.status, TF_DEV_BAD_PAGE);
-                } else {
-                    bytes += (uint32_t)(BR * 128 * C::kSlabs);
-                }
+    if (warp == 4) {
+        // ================= issuer warp: every lane walks the tiles; lane 0
+        // issues the MMAs, and the TMA boxes of a tile go out one per lane, so
+        // one warp instruction issues all of them
+        {
+            if (lane == 0) {
+                prefetch_tensormap(&tmQ);
+                prefetch_tensormap(&tmK);
+                prefetch_tensormap(&tmV);
             }
-            pid[b] = id;
-        }
-        mbar_arrive_expect_tx(bar, bytes);
-        for (int b = 0; b < n_box; ++b) {
-            if (pid[b] < 0) continue;
-            const int key0 = kt + b * BR;
-            for (int s = 0; s < C::kSlabs; ++s)
-                tma_load_4d(dst0 + s * kSlabBytes + b * BR * 128, map, bar, 64 * s, key0 & (P - 1), g, pid[b]);
-        }
-    };
-
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bq, (uint32_t)C::kTileBytes);
-        for (int s = 0; s < C::kSlabs; ++s) tma_load_3d(sQ + s * kSlabBytes, &tmQ, bq, 64 * s, g * G, p.q_row + row0);
-        if (n_tiles > 0) {
-            issue_kv(0, false);
-            issue_kv(0, true);
-        }
-    }
-
-    // this thread's query
-    const int qi = tid;
-    const int row_i = row0 + qi / G;  // chunk-relative
-    const bool valid_row = row_i < T;
-    const int lim = valid_row ? (N - T + row_i + 1) : key_hi_eff;
-    const float scale_log2 = p.scale_log2;
-    float m_ref = -INFINITY, l_run = 0.f;
-    uint32_t emax = 0, tail_bad = 0, timed_out = 0;
-
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t idesc_qk = umma_idesc_bf16(128, kBN, false, false);
-    const uint32_t idesc_pv = umma_idesc_bf16(128, D, false, true);
-
-    for (int t = 0; t < n_tiles; ++t) {
-        const int kt = t * kBN;
-        const uint32_t ph = (uint32_t)(t & 1);
-        // ---- S = Q K^T
-        if (!mbar_wait(bk, ph)) timed_out = 1;
-        if (t == 0 && !mbar_wait(bq, 0)) timed_out = 1;
-        if (__syncthreads_or(timed_out)) break;
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-                const int s = k >> 2, kk = k & 3;
-                const uint64_t ad = umma_desc_sw128(sQ + s * kSlabBytes + kk * 32, 16, 1024);
-                const uint64_t bd = umma_desc_sw128(sK + s * kSlabBytes + kk * 32, 16, 1024);
-                umma_ss(tmem + kColS, ad, bd, idesc_qk, k > 0 ? 1u : 0u);
-            }
-            umma_commit(bs);
-        }
-        if (!mbar_wait(bs, ph)) timed_out = 1;
-        if (__syncthreads_or(timed_out)) break;
-        tc_fence_after();
-        if (tid == 0 && t + 1 < n_tiles) issue_kv(t + 1, false);  // the K buffer is free again
-
-        // ---- softmax over this thread's row
-        float sv[kBN];
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(lane_base + kColS + c * 32, r);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(r[j]);
-        }
-        tmem_wait_ld();
-        const bool need_mask = kt + kBN > full_hi;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-            float x = sv[c] * scale_log2;
-            const bool vis = !need_mask || (kt + c < lim);
-            emax = max(emax, vis ? exp_bits(x) : 0u);
-            x = vis ? x : -INFINITY;
-            sv[c] = x;
-            mx = fmaxf(mx, x);
-        }
-        float alpha = 1.f;
-        if (mx > m_ref + 8.f || (m_ref == -INFINITY && mx != -INFINITY)) {
-            alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
-            m_ref = mx;
-        }
-        const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float ls = 0.f;
-#pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) {
-            uint32_t hi[16], lo[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float p0 = ex2(sv[c * 32 + 2 * j] - mu), p1 = ex2(sv[c * 32 + 2 * j + 1] - mu);
-                ls += p0 + p1;
-                hi[j] = pack_bf16x2(p0, p1);
-                lo[j] = pack_bf16x2(p0 - bf16_lo_to_f32(hi[j]), p1 - bf16_hi_to_f32(hi[j]));
-            }
-            tmem_st16(lane_base + kColPhi + c * 16, hi);
-            tmem_st16(lane_base + kColPlo + c * 16, lo);
-        }
-        l_run = l_run * alpha + ls;
-        // rescale O when this row's reference max moved (O holds the previous tiles)
-        if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(lane_base + kColO + c * 32, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                tmem_st32(lane_base + kColO + c * 32, r);
-            }
-        }
-        tmem_wait_st();
-
-        // ---- V: wait, then clean the rows this tile must not feed into P V
-        if (!mbar_wait(bv, ph)) timed_out = 1;
-        if (__syncthreads_or(timed_out)) break;
-        if (kt + kBN > full_hi) {
-            // rows past every valid row's keys: zero; rows only some rows see: zero if nonfinite
-            for (int idx = tid; idx < kBN * C::kSlabs; idx += kPTThreads) {
-                const int r = idx % kBN, s = idx / kBN;
-                const int key = kt + r;
-                uint4 *rowp = reinterpret_cast<uint4 *>(sbase_ptr + 2 * C::kTileBytes + s * kSlabBytes + r * 128);
-                if (key >= key_hi_eff) {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
-                } else if (key >= full_hi) {
-                    bool nf = false;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint4 v = rowp[k];
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            nf |= ((w[e] & 0x7f80u) == 0x7f80u) || ((w[e] & 0x7f800000u) == 0x7f800000u);
+            const int n_copies = n_box * C::kSlabs;  // boxes of one K (or V) tile, <= 32
+            // every lane waits; the answer is the warp's, so all lanes branch alike
+            auto wwait = [&](uint32_t bar, uint32_t phase, volatile uint32_t *ab) {
+                return __all_sync(0xffffffffu, pt_wait(bar, phase, ab));
+            };
+            // K or V tile t into buffer t & 1: one box per page (or per 64-key span
+            // of a larger page) and 64-column slab; page ids come from shared memory
+            auto issue_kv = [&](int t, bool is_v) {
+                const int kt = t * kBN, b = t & 1;
+                const uint32_t dst0 = is_v ? sV(b) : sK(b);
+                const uint32_t bar = is_v ? bv(b) : bk(b);
+                const CUtensorMap *map = is_v ? &tmV : &tmK;
+                // lane i < n_copies owns box x = i / slabs, slab sl = i % slabs
+                const int x = lane / C::kSlabs, sl = lane % C::kSlabs;
+                const int key0 = kt + x * BR;
+                int id = -1;
+                if (lane < n_copies && key0 < key_hi_eff) {
+                    const int idx = key0 >> p.log2_page;
+                    if (idx >= p.n_pg)
+                        id = -2;
+                    else if (idx < C::kPidCap)
+                        id = pids[idx];
+                    else  // past the shared-memory copy (very long prompts with small pages)
+                        id = p.page_table[p.pt_base + idx];
+                    if (id < 0 || id >= p.n_pages) {
+                        id = -1;
+                        s_err = 1;
+                        atomicOr(p.status, TF_DEV_BAD_PAGE);
                     }
-                    if (nf) atomicOr(&s_vbad[r >> 5], 1u << (r & 31));
+                }
+                const uint32_t live = __ballot_sync(0xffffffffu, id >= 0);
+                if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)__popc(live) * (uint32_t)(BR * 128));
+                __syncwarp();
+                if (id >= 0) tma_load_4d(dst0 + sl * kKVSlab + x * BR * 128, map, bar, 64 * sl, key0 & (P - 1), g, id);
+            };
+            const uint32_t idesc_qk = umma_idesc_bf16(kQM, kBN, false, false);
+            const uint32_t idesc_pv = umma_idesc_bf16(kQM, D, false, true);
+            auto issue_qk = [&](int t) {
+                if (lane == 0) {
+                    const int b = t & 1;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const int sl = k >> 2, kk = k & 3;
+                        const uint64_t ad = umma_desc_sw128(sQ + sl * kQSlab + kk * 32, 16, 1024);
+                        const uint64_t bd = umma_desc_sw128(sK(b) + sl * kKVSlab + kk * 32, 16, 1024);
+                        umma_ss(tmem + (b ? kColS1 : kColS0), ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bsq(b));
+                }
+                __syncwarp();
+            };
+
+            if (lane == 0) mbar_arrive_expect_tx(bq, (uint32_t)C::kQBytes);
+            __syncwarp();
+            if (lane < C::kSlabs) tma_load_3d(sQ + lane * kQSlab, &tmQ, bq, 64 * lane, g * G, p.q_row + row0);
+            for (int t = 0; t < 2 && t < n_tiles; ++t) {
+                issue_kv(t, false);
+                issue_kv(t, true);
+            }
+            if (n_tiles > 0 && wwait(bq, 0, abort_flag) && wwait(bk(0), 0, abort_flag)) issue_qk(0);
+            for (int j = 0; j < n_tiles; ++j) {
+                const int b = j & 1;
+                const uint32_t ph = (uint32_t)((j >> 1) & 1);
+                // the next tile's scores while the softmax warps work on this one;
+                // its S buffer held P(j-1), whose P V was issued before (in order)
+                if (j + 1 < n_tiles && wwait(bk((j + 1) & 1), (uint32_t)(((j + 1) >> 1) & 1), abort_flag))
+                    issue_qk(j + 1);
+                // QK(j) done: its K buffer takes tile j + 2
+                if (j + 2 < n_tiles && wwait(bsq(b), ph, abort_flag)) issue_kv(j + 2, false);
+                // P(j) written (and V(j) cleaned) and V(j) landed: O += P V
+                const bool ok = wwait(bpr(b), ph, abort_flag) && wwait(bv(b), ph, abort_flag);
+                if (ok && lane == 0) {
+                    tc_fence_after();
+                    const uint32_t sb = tmem + (b ? kColS1 : kColS0);
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        const uint64_t bd = umma_desc_sw128(sV(b) + kk * 16 * 128, kKVSlab, 1024);
+                        umma_ts(tmem + kColO, sb + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                        if (HILO) umma_ts(tmem + kColO, sb + 32 + kk * 8, bd, idesc_pv, 1u);
+                    }
+                    umma_commit(bo(b));
+                }
+                __syncwarp();
+                // P V(j-1) done: its V buffer takes tile j + 1
+                if (j >= 1 && j + 1 < n_tiles &&
+                    wwait(bo((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag))
+                    issue_kv(j + 1, true);
+            }
+        }
+    } else {
+        // ================= softmax warps: thread tid owns query row tid
+        const int qi = tid;
+        const int row_i = row0 + qi / G;  // chunk-relative
+        const bool valid_row = row_i < T;
+        const int lim = valid_row ? (N - T + row_i + 1) : key_hi_eff;
+        const float scale_log2 = p.scale_log2;
+        float m_ref = -INFINITY, l_run = 0.f;
+        uint32_t emax = 0, tail_bad = 0;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+
+        for (int j = 0; j < n_tiles; ++j) {
+            const int b = j & 1, kt = j * kBN;
+            const uint32_t ph = (uint32_t)((j >> 1) & 1);
+            const uint32_t colS = b ? kColS1 : kColS0;
+            pt_wait(bsq(b), ph, abort_flag);
+            tc_fence_after();
+            float sv[kBN];
+            {
+                uint32_t r[32];
+                tmem_ld32(lane_base + colS, r);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sv[c] = __uint_as_float(r[c]);
+                tmem_ld32(lane_base + colS + 32, r);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sv[32 + c] = __uint_as_float(r[c]);
+            }
+            tmem_wait_ld();
+            const bool need_mask = kt + kBN > full_hi;
+            // the tile's largest score; nonfinite visible scores: NaN and +inf
+            // reach the row sum (checked at the end), -inf is caught by the min
+            float mx = -INFINITY;
+            if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) {
+                    const bool vis = kt + c < lim;
+                    emax = max(emax, vis ? exp_bits(sv[c]) : 0u);
+                    sv[c] = vis ? sv[c] : -INFINITY;
+                    mx = fmaxf(mx, sv[c]);
+                }
+            } else {
+                float mn = INFINITY;
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) {
+                    mx = fmaxf(mx, sv[c]);
+                    mn = fminf(mn, sv[c]);
+                }
+                if (mn == -INFINITY) emax = 0x7f800000u;
+            }
+            mx *= scale_log2;  // scale > 0: the max commutes with it
+            // lazy rescale: the reference max moves only when it rises by 2^8
+            float alpha = 1.f;
+            if (mx > m_ref + 8.f || (m_ref == -INFINITY && mx != -INFINITY)) {
+                alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+                m_ref = mx;
+            }
+            const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+            {
+                uint32_t hi[32];
+                float ls = 0.f;
+                if constexpr (HILO) {
+                    uint32_t lo[32];
+#pragma unroll
+                    for (int w = 0; w < 32; ++w) {
+                        const float p0 = ex2(fmaf(sv[2 * w], scale_log2, -mu));
+                        const float p1 = ex2(fmaf(sv[2 * w + 1], scale_log2, -mu));
+                        ls += p0 + p1;
+                        hi[w] = pack_bf16x2(p0, p1);
+                        lo[w] = pack_bf16x2(p0 - bf16_lo_to_f32(hi[w]), p1 - bf16_hi_to_f32(hi[w]));
+                    }
+                    tmem_st32(lane_base + colS + 32, lo);
+                } else {
+#pragma unroll
+                    for (int w = 0; w < 32; ++w) {
+                        const float p0 = ex2(fmaf(sv[2 * w], scale_log2, -mu));
+                        const float p1 = ex2(fmaf(sv[2 * w + 1], scale_log2, -mu));
+                        ls += p0 + p1;
+                        hi[w] = pack_bf16x2(p0, p1);
+                    }
+                }
+                l_run = l_run * alpha + ls;
+                tmem_st32(lane_base + colS, hi);
+            }
+            // O holds the tiles before this one: rescale it once P V(j-1) is done
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                pt_wait(bo((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag);
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(lane_base + kColO + c * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int w = 0; w < 32; ++w) r[w] = __float_as_uint(__uint_as_float(r[w]) * alpha);
+                    tmem_st32(lane_base + kColO + c * 32, r);
                 }
             }
-            __syncthreads();
-            const uint32_t vb[4] = {s_vbad[0], s_vbad[1], s_vbad[2], s_vbad[3]};
-            if (vb[0] | vb[1] | vb[2] | vb[3]) {
-                for (int idx = tid; idx < kBN * C::kSlabs; idx += kPTThreads) {
-                    const int r = idx % kBN, s = idx / kBN;
-                    if ((vb[r >> 5] >> (r & 31)) & 1u) {
-                        uint4 *rowp =
-                            reinterpret_cast<uint4 *>(sbase_ptr + 2 * C::kTileBytes + s * kSlabBytes + r * 128);
+            tmem_wait_st();
+            // V rows this tile must not feed into P V: past every row's keys ->
+            // zero; seen by only some rows and nonfinite -> zero and flag
+            if (kt + kBN > full_hi) {
+                pt_wait(bv(b), ph, abort_flag);
+                named_bar_sync(1, kPTSoftmax);
+                if (tid == 0) s_vbad[0] = s_vbad[1] = 0;
+                named_bar_sync(1, kPTSoftmax);
+                unsigned char *vb = sbase_ptr + C::kOffV + b * C::kKVBytes;
+                for (int idx = tid; idx < kBN * C::kSlabs; idx += kPTSoftmax) {
+                    const int r = idx % kBN, sl = idx / kBN;
+                    uint4 *rowp = reinterpret_cast<uint4 *>(vb + sl * kKVSlab + r * 128);
+                    const int key = kt + r;
+                    if (key >= key_hi_eff) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
+                    } else if (key >= full_hi) {
+                        bool nf = false;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint4 v = rowp[k];
+                            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                nf |= ((w4[e] & 0x7f80u) == 0x7f80u) || ((w4[e] & 0x7f800000u) == 0x7f800000u);
+                        }
+                        if (nf) atomicOr(&s_vbad[r >> 5], 1u << (r & 31));
                     }
                 }
-                for (int r = 0; r < kBN; ++r)
-                    if (((vb[r >> 5] >> (r & 31)) & 1u) && kt + r < lim) tail_bad = 1;
-            }
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (tid == 0) s_vbad[0] = s_vbad[1] = s_vbad[2] = s_vbad[3] = 0;
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- O += P V (A = P from tensor memory, B = V MN-major)
-        if (tid == 0) {
-            tc_fence_after();
+                named_bar_sync(1, kPTSoftmax);
+                const uint32_t vb0 = s_vbad[0], vb1 = s_vbad[1];
+                if (vb0 | vb1) {
+                    for (int idx = tid; idx < kBN * C::kSlabs; idx += kPTSoftmax) {
+                        const int r = idx % kBN, sl = idx / kBN;
+                        if ((((r < 32) ? vb0 : vb1) >> (r & 31)) & 1u) {
+                            uint4 *rowp = reinterpret_cast<uint4 *>(vb + sl * kKVSlab + r * 128);
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-                const uint64_t bd = umma_desc_sw128(sV + kk * 16 * 128, kSlabBytes, 1024);
-                umma_ts(tmem + kColO, tmem + kColPhi + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-                umma_ts(tmem + kColO, tmem + kColPlo + kk * 8, bd, idesc_pv, 1u);
+                            for (int k = 0; k < 8; ++k) rowp[k] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    for (int r = 0; r < kBN; ++r)
+                        if (((((r < 32) ? vb0 : vb1) >> (r & 31)) & 1u) && kt + r < lim) tail_bad = 1;
+                }
+                fence_proxy_async_smem();
             }
-            umma_commit(bo);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bpr(b));
         }
-        if (!mbar_wait(bo, ph)) timed_out = 1;
-        if (__syncthreads_or(timed_out)) break;
-        tc_fence_after();
-        if (tid == 0 && t + 1 < n_tiles) issue_kv(t + 1, true);  // the V buffer is free again
-    }
 
-    // ---- epilogue: O / l, nonfinite check, store
-    timed_out = __syncthreads_or(timed_out) ? 1u : 0u;  // uniform over the CTA
-    if (timed_out) {
-        // give in-flight copies and MMAs a bounded chance to land before the
-        // tensor memory is released
-        if (tid == 0) report_timeout(p.status);
-        for (int i = 0; i < 2; ++i) {
-            mbar_wait(bk, (uint32_t)i, 20000000ull);
-            mbar_wait(bv, (uint32_t)i, 20000000ull);
-            mbar_wait(bs, (uint32_t)i, 20000000ull);
-            mbar_wait(bo, (uint32_t)i, 20000000ull);
-        }
-    }
-    uint32_t bad = (emax == 0x7f800000u) | tail_bad | (uint32_t)s_err | timed_out;
-    if (!(l_run > 0.f) || !isfinite(l_run)) bad = 1;
-    const int64_t u = (int64_t)(p.q_row + row_i) * p.hq + g * G + (qi % G);
-    if (!timed_out) {
+        // ---- epilogue: O / l, nonfinite check, store
+        if (n_tiles > 0) pt_wait(bo((n_tiles - 1) & 1), (uint32_t)(((n_tiles - 1) >> 1) & 1), abort_flag);
+        tc_fence_after();
+        const bool aborted = *abort_flag != 0;
+        uint32_t bad = (emax == 0x7f800000u) | tail_bad | s_err | (aborted ? 1u : 0u);
+        if (!(l_run > 0.f) || !isfinite(l_run)) bad = 1;
+        const int64_t u = (int64_t)(p.q_row + row_i) * p.hq + g * G + (qi % G);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
@@ -320,41 +390,53 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             tmem_wait_ld();
             float o[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                o[j] = __uint_as_float(r[j]) / l_run;
-                bad |= !isfinite(o[j]);
+            for (int w = 0; w < 32; ++w) {
+                o[w] = __uint_as_float(r[w]) / l_run;
+                bad |= !isfinite(o[w]);
             }
-            if (valid_row) {
+            if (valid_row && !aborted) {
                 if (p.out_bf16) {
                     uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + c * 32);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dst[j] = make_uint4(pack_bf16x2(o[8 * j], o[8 * j + 1]), pack_bf16x2(o[8 * j + 2], o[8 * j + 3]),
-                                            pack_bf16x2(o[8 * j + 4], o[8 * j + 5]),
-                                            pack_bf16x2(o[8 * j + 6], o[8 * j + 7]));
+                    for (int w = 0; w < 4; ++w)
+                        dst[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]), pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
+                                            pack_bf16x2(o[8 * w + 4], o[8 * w + 5]),
+                                            pack_bf16x2(o[8 * w + 6], o[8 * w + 7]));
                 } else {
                     float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + c * 32);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) dst[j] = make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                    for (int w = 0; w < 8; ++w) dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
                 }
             }
+        }
+        if (valid_row) {
+            if (bad) {
+                const float qnan = __int_as_float(0x7fc00000);
+                for (int d = 0; d < D; d += 8) {
+                    if (p.out_bf16)
+                        *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d) =
+                            make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
+                    else {
+                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d);
+                        dst[0] = make_float4(qnan, qnan, qnan, qnan);
+                        dst[1] = make_float4(qnan, qnan, qnan, qnan);
+                    }
+                }
+            }
+            if (p.out_flags) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
         }
     }
-    if (valid_row) {
-        if (bad) {
-            const float qnan = __int_as_float(0x7fc00000);
-            for (int d = 0; d < D; d += 8) {
-                if (p.out_bf16)
-                    *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d) =
-                        make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
-                else {
-                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d);
-                    dst[0] = make_float4(qnan, qnan, qnan, qnan);
-                    dst[1] = make_float4(qnan, qnan, qnan, qnan);
-                }
+    // everyone: report a timeout, give in-flight work a bounded chance to land,
+    // release tensor memory
+    __syncthreads();
+    if (s_abort) {
+        if (tid == 0) atomicOr(p.status, TF_DEV_TIMEOUT);
+        if (tid == 0)
+            for (int i = 0; i < 11; ++i) {
+                mbar_wait(smem_u32(&bars[i]), 0u, 20000000ull);
+                mbar_wait(smem_u32(&bars[i]), 1u, 20000000ull);
             }
-        }
-        if (p.out_flags) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
+        __syncthreads();
     }
     tc_fence_before();
     __syncthreads();
@@ -377,7 +459,7 @@ template <int D>
 static cudaError_t launch_prompt_tc_t(const PromptTcParams &p, const void *q, const void *k, const void *v,
                                       cudaStream_t st) {
     CUtensorMap mq, mk, mv;
-    const int G = p.group, RT = 128 / G, P = 1 << p.log2_page, BR = P < 128 ? P : 128;
+    const int G = p.group, RT = kQM / G, P = 1 << p.log2_page, BR = P < kBN ? P : kBN;
     {
         const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.hq, (cuuint64_t)p.n_rows_total};
         const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.hq * D * 2};
@@ -391,7 +473,7 @@ static cudaError_t launch_prompt_tc_t(const PromptTcParams &p, const void *q, co
         if (!make_tensor_map_bf16(&mk, k, 4, dims, strides, box)) return cudaErrorInvalidValue;
         if (!make_tensor_map_bf16(&mv, v, 4, dims, strides, box)) return cudaErrorInvalidValue;
     }
-    auto kern = prompt_tc_kernel<D>;
+    auto kern = p.out_bf16 ? prompt_tc_kernel<D, false> : prompt_tc_kernel<D, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PTCfg<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((p.n_rows + RT - 1) / RT), (unsigned)p.hkv);

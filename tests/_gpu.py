@@ -124,3 +124,36 @@ def compare_attn(gpu_out, gpu_flags, orc_out, orc_flags, sel=None, max_abs=MAX_A
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
     ax = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
     return np.exp2(np.floor(np.log2(ax)) - 7)
+
+
+# bf16-output prompt tolerance, derived from the arithmetic: the softmax
+# weights enter the P.V product as bf16 (relative error <= 2^-9 each), so the
+# fp32 sum is off by at most 2^-9 * max_j |V_jd|; rounding the output to bf16
+# adds at most 2^-9 * |out|.  A factor 2 covers fp32 accumulation.  The
+# relative L2 bound (3e-3) is about twice the rms the two roundings give.
+PROMPT_BF16_REL_L2 = 3e-3
+
+
+def prompt_bf16_bound(b, ref):
+    """Per-element bound [rows][Hq][D] for a one-stream prompt batch."""
+    n = int(b.segs[0][2])
+    p = b.page_size
+    pages = b.page_table[b.segs[0][3]: b.segs[0][3] + -(-n // p)]
+    v = wl.bf16_bits_to_f32(b.v_pool[pages]).astype(np.float64)  # [pages][Hkv][P][D]
+    v = v.transpose(1, 0, 2, 3).reshape(b.n_kv_heads, -1, b.head_dim)[:, :n]  # [Hkv][n][D]
+    vmax = np.nanmax(np.abs(v), axis=1)  # [Hkv][D]
+    g = np.arange(b.n_q_heads) // (b.n_q_heads // b.n_kv_heads)
+    return 2.0 ** -8 * (vmax[g][None, :, :] + np.abs(ref))
+
+
+def check_prompt_bf16(gpu, gflags, ref, rflags, bound, sel=None, what="prompt bf16"):
+    if sel is None:
+        sel = np.ones(rflags.shape, bool)
+    np.testing.assert_array_equal(gflags[sel], rflags[sel], err_msg=f"{what}: flags differ")
+    ok = sel & ~rflags.astype(bool)
+    if (sel & rflags.astype(bool)).any():
+        assert np.isnan(gpu[sel & rflags.astype(bool)]).all()
+    err = np.abs(gpu[ok].astype(np.float64) - ref[ok])
+    assert (err <= bound[ok]).all(), f"{what}: beyond the derived bound by {np.max(err - bound[ok]):.3e}"
+    rl2 = np.linalg.norm(gpu[ok] - ref[ok]) / np.linalg.norm(ref[ok])
+    assert rl2 <= PROMPT_BF16_REL_L2, f"{what}: rel-L2 {rl2:.3e}"
