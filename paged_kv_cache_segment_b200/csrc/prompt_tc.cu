@@ -7,22 +7,27 @@
 // pages of 32); review thread: the per-chunk page lookup is hoisted out of the
 // key loop.
 //
-// One CTA of four warps computes 128 queries: 128/G consecutive rows x the G
-// q-heads that share kv-head g, so one K/V tile serves all of them.  Per
-// 128-key tile:
-//   1. TMA brings K (and V) in 128-byte-swizzled 64-column slabs; page ids are
-//      resolved once per tile (a box per page), so no lookup sits in any
-//      inner loop;
-//   2. one thread issues S = Q K^T (M 128, N 128, K = D) into tensor memory;
-//   3. every thread owns one query row: it loads its S row from tensor memory,
-//      masks it causally, and folds it into a running max / sum with a lazy
-//      rescale (the reference max moves only when it rises by more than 2^8);
+// One CTA computes 128 queries: 128/G consecutive rows x the G q-heads that
+// share kv-head g, so one K/V tile serves all of them.  Six warps split the
+// work by role: a TMA warp, an MMA warp and four softmax warps.  Per 64-key
+// tile:
+//   1. the TMA warp brings K (and V) in 128-byte-swizzled 64-column slabs, one
+//      box per page (or per 64-key span of a larger page) and slab, every lane
+//      issuing one box; the CTA's page ids were copied to shared memory once,
+//      so no page-table read sits in the key loop;
+//   2. the MMA warp issues S = Q K^T (M 128, N 64, K = D) into tensor memory,
+//      one tile ahead of the softmax (two S buffers);
+//   3. every softmax thread owns one query row: it loads its S row from tensor
+//      memory, masks it causally, and folds it into a running max / sum with a
+//      lazy rescale (the reference max moves only when it rises by 2^8);
 //   4. the weights go back to tensor memory (into the S columns they came
-//      from) and one thread issues O += P V (A from tensor memory, B = V in
+//      from) and the MMA warp issues O += P V (A from tensor memory, B = V in
 //      shared memory, MN-major).  For f32 output P is fed as bf16 hi + bf16 lo
 //      (two MMAs, about 16 bits a weight, so the fp32 tolerance holds); for
 //      bf16 output P is one bf16, whose rounding is below the output's own;
 //   5. O stays in tensor memory until the epilogue divides by the sum.
+// K and V each have two buffers; a buffer is refilled as soon as the MMA that
+// read it has completed.
 // Nonfinite handling matches the other attention kernels: visible scores are
 // checked through their exponent bits, value rows that only some rows see
 // are scanned and zeroed, and the final O and sum are checked.
@@ -38,7 +43,7 @@
 namespace tfp {
 
 constexpr int kPTSoftmax = 128;               // four softmax warps, one query row a thread
-constexpr int kPTThreads = kPTSoftmax + 32;   // + one issuer warp (MMAs and TMA)
+constexpr int kPTThreads = kPTSoftmax + 64;   // + an MMA warp and a TMA warp
 constexpr int kQM = 128;                      // queries a CTA (the MMA's M)
 constexpr int kBN = 64;                       // keys a tile
 constexpr int kQSlab = kQM * 128;             // 128 query rows x 128 bytes
@@ -129,105 +134,100 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     tc_fence_after();
     const uint32_t tmem = s_tmem;
 
-    if (warp == 4) {
-        // ================= issuer warp: every lane walks the tiles; lane 0
-        // issues the MMAs, and the TMA boxes of a tile go out one per lane, so
-        // one warp instruction issues all of them
-        {
-            if (lane == 0) {
-                prefetch_tensormap(&tmQ);
-                prefetch_tensormap(&tmK);
-                prefetch_tensormap(&tmV);
+    // every lane of a helper warp waits; the answer is the warp's, so all lanes branch alike
+    auto wwait = [&](uint32_t bar, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(bar, phase, abort_flag)); };
+    if (warp == 5) {
+        // ================= TMA warp: the K/V boxes of a tile go out one per lane,
+        // so one warp instruction issues all of them; a buffer is refilled as
+        // soon as the MMA that read it is done
+        if (lane == 0) {
+            prefetch_tensormap(&tmQ);
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+        }
+        const int n_copies = n_box * C::kSlabs;  // boxes of one K (or V) tile, <= 32
+        // K or V tile t into buffer t & 1: one box per page (or per 64-key span
+        // of a larger page) and 64-column slab; page ids come from shared memory
+        auto issue_kv = [&](int t, bool is_v) {
+            const int kt = t * kBN, b = t & 1;
+            const uint32_t dst0 = is_v ? sV(b) : sK(b);
+            const uint32_t bar = is_v ? bv(b) : bk(b);
+            const CUtensorMap *map = is_v ? &tmV : &tmK;
+            // lane i < n_copies owns box x = i / slabs, slab sl = i % slabs
+            const int x = lane / C::kSlabs, sl = lane % C::kSlabs;
+            const int key0 = kt + x * BR;
+            int id = -1;
+            if (lane < n_copies && key0 < key_hi_eff) {
+                const int idx = key0 >> p.log2_page;
+                if (idx >= p.n_pg)
+                    id = -2;
+                else if (idx < C::kPidCap)
+                    id = pids[idx];
+                else  // past the shared-memory copy (very long prompts with small pages)
+                    id = p.page_table[p.pt_base + idx];
+                if (id < 0 || id >= p.n_pages) {
+                    id = -1;
+                    s_err = 1;
+                    atomicOr(p.status, TF_DEV_BAD_PAGE);
+                }
             }
-            const int n_copies = n_box * C::kSlabs;  // boxes of one K (or V) tile, <= 32
-            // every lane waits; the answer is the warp's, so all lanes branch alike
-            auto wwait = [&](uint32_t bar, uint32_t phase, volatile uint32_t *ab) {
-                return __all_sync(0xffffffffu, pt_wait(bar, phase, ab));
-            };
-            // K or V tile t into buffer t & 1: one box per page (or per 64-key span
-            // of a larger page) and 64-column slab; page ids come from shared memory
-            auto issue_kv = [&](int t, bool is_v) {
-                const int kt = t * kBN, b = t & 1;
-                const uint32_t dst0 = is_v ? sV(b) : sK(b);
-                const uint32_t bar = is_v ? bv(b) : bk(b);
-                const CUtensorMap *map = is_v ? &tmV : &tmK;
-                // lane i < n_copies owns box x = i / slabs, slab sl = i % slabs
-                const int x = lane / C::kSlabs, sl = lane % C::kSlabs;
-                const int key0 = kt + x * BR;
-                int id = -1;
-                if (lane < n_copies && key0 < key_hi_eff) {
-                    const int idx = key0 >> p.log2_page;
-                    if (idx >= p.n_pg)
-                        id = -2;
-                    else if (idx < C::kPidCap)
-                        id = pids[idx];
-                    else  // past the shared-memory copy (very long prompts with small pages)
-                        id = p.page_table[p.pt_base + idx];
-                    if (id < 0 || id >= p.n_pages) {
-                        id = -1;
-                        s_err = 1;
-                        atomicOr(p.status, TF_DEV_BAD_PAGE);
-                    }
-                }
-                const uint32_t live = __ballot_sync(0xffffffffu, id >= 0);
-                if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)__popc(live) * (uint32_t)(BR * 128));
-                __syncwarp();
-                if (id >= 0) tma_load_4d(dst0 + sl * kKVSlab + x * BR * 128, map, bar, 64 * sl, key0 & (P - 1), g, id);
-            };
-            const uint32_t idesc_qk = umma_idesc_bf16(kQM, kBN, false, false);
-            const uint32_t idesc_pv = umma_idesc_bf16(kQM, D, false, true);
-            auto issue_qk = [&](int t) {
-                if (lane == 0) {
-                    const int b = t & 1;
-                    tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k) {
-                        const int sl = k >> 2, kk = k & 3;
-                        const uint64_t ad = umma_desc_sw128(sQ + sl * kQSlab + kk * 32, 16, 1024);
-                        const uint64_t bd = umma_desc_sw128(sK(b) + sl * kKVSlab + kk * 32, 16, 1024);
-                        umma_ss(tmem + (b ? kColS1 : kColS0), ad, bd, idesc_qk, k > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bsq(b));
-                }
-                __syncwarp();
-            };
-
-            if (lane == 0) mbar_arrive_expect_tx(bq, (uint32_t)C::kQBytes);
+            const uint32_t live = __ballot_sync(0xffffffffu, id >= 0);
+            if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)__popc(live) * (uint32_t)(BR * 128));
             __syncwarp();
-            if (lane < C::kSlabs) tma_load_3d(sQ + lane * kQSlab, &tmQ, bq, 64 * lane, g * G, p.q_row + row0);
-            for (int t = 0; t < 2 && t < n_tiles; ++t) {
-                issue_kv(t, false);
-                issue_kv(t, true);
-            }
-            if (n_tiles > 0 && wwait(bq, 0, abort_flag) && wwait(bk(0), 0, abort_flag)) issue_qk(0);
-            for (int j = 0; j < n_tiles; ++j) {
-                const int b = j & 1;
-                const uint32_t ph = (uint32_t)((j >> 1) & 1);
-                // the next tile's scores while the softmax warps work on this one;
-                // its S buffer held P(j-1), whose P V was issued before (in order)
-                if (j + 1 < n_tiles && wwait(bk((j + 1) & 1), (uint32_t)(((j + 1) >> 1) & 1), abort_flag))
-                    issue_qk(j + 1);
-                // QK(j) done: its K buffer takes tile j + 2
-                if (j + 2 < n_tiles && wwait(bsq(b), ph, abort_flag)) issue_kv(j + 2, false);
-                // P(j) written (and V(j) cleaned) and V(j) landed: O += P V
-                const bool ok = wwait(bpr(b), ph, abort_flag) && wwait(bv(b), ph, abort_flag);
-                if (ok && lane == 0) {
-                    tc_fence_after();
-                    const uint32_t sb = tmem + (b ? kColS1 : kColS0);
+            if (id >= 0) tma_load_4d(dst0 + sl * kKVSlab + x * BR * 128, map, bar, 64 * sl, key0 & (P - 1), g, id);
+        };
+        if (lane == 0) mbar_arrive_expect_tx(bq, (uint32_t)C::kQBytes);
+        __syncwarp();
+        if (lane < C::kSlabs) tma_load_3d(sQ + lane * kQSlab, &tmQ, bq, 64 * lane, g * G, p.q_row + row0);
+        for (int t = 0; t < n_tiles; ++t) {
+            const int pb = (t - 2) & 1;
+            const uint32_t pph = (uint32_t)(((t - 2) >> 1) & 1);
+            // K(t) once QK(t-2) has read the buffer, V(t) once P V(t-2) has
+            if (t >= 2 && !wwait(bsq(pb), pph)) break;
+            issue_kv(t, false);
+            if (t >= 2 && !wwait(bo(pb), pph)) break;
+            issue_kv(t, true);
+        }
+    } else if (warp == 4) {
+        // ================= MMA warp: lane 0 issues every tcgen05.mma
+        const uint32_t idesc_qk = umma_idesc_bf16(kQM, kBN, false, false);
+        const uint32_t idesc_pv = umma_idesc_bf16(kQM, D, false, true);
+        auto issue_qk = [&](int t) {
+            if (lane == 0) {
+                const int b = t & 1;
+                tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        const uint64_t bd = umma_desc_sw128(sV(b) + kk * 16 * 128, kKVSlab, 1024);
-                        umma_ts(tmem + kColO, sb + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                        if (HILO) umma_ts(tmem + kColO, sb + 32 + kk * 8, bd, idesc_pv, 1u);
-                    }
-                    umma_commit(bo(b));
+                for (int k = 0; k < D / 16; ++k) {
+                    const int sl = k >> 2, kk = k & 3;
+                    const uint64_t ad = umma_desc_sw128(sQ + sl * kQSlab + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(sK(b) + sl * kKVSlab + kk * 32, 16, 1024);
+                    umma_ss(tmem + (b ? kColS1 : kColS0), ad, bd, idesc_qk, k > 0 ? 1u : 0u);
                 }
-                __syncwarp();
-                // P V(j-1) done: its V buffer takes tile j + 1
-                if (j >= 1 && j + 1 < n_tiles &&
-                    wwait(bo((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag))
-                    issue_kv(j + 1, true);
+                umma_commit(bsq(b));
             }
+            __syncwarp();
+        };
+        if (n_tiles > 0 && wwait(bq, 0) && wwait(bk(0), 0)) issue_qk(0);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int b = j & 1;
+            const uint32_t ph = (uint32_t)((j >> 1) & 1);
+            // the next tile's scores while the softmax warps work on this one;
+            // its S buffer held P(j-1), whose P V was issued before (in order)
+            if (j + 1 < n_tiles && wwait(bk((j + 1) & 1), (uint32_t)(((j + 1) >> 1) & 1))) issue_qk(j + 1);
+            // P(j) written (and V(j) cleaned) and V(j) landed: O += P V
+            const bool ok = wwait(bpr(b), ph) && wwait(bv(b), ph);
+            if (ok && lane == 0) {
+                tc_fence_after();
+                const uint32_t sb = tmem + (b ? kColS1 : kColS0);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    const uint64_t bd = umma_desc_sw128(sV(b) + kk * 16 * 128, kKVSlab, 1024);
+                    umma_ts(tmem + kColO, sb + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    if (HILO) umma_ts(tmem + kColO, sb + 32 + kk * 8, bd, idesc_pv, 1u);
+                }
+                umma_commit(bo(b));
+            }
+            __syncwarp();
         }
     } else {
         // ================= softmax warps: thread tid owns query row tid
