@@ -328,7 +328,7 @@ def run_native(args):
         "config": {"workload": WORKLOAD, "streams": 16, "kv_bytes_per_step": kv_bytes,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2: 3 rotating copies of the batch (906 MB of KV), step k reads copy k % 3"},
-        "roofline": roofline("hbm", achieved, peaks["hbm_gbs"], "GB/s", traffic.get("decode_partial_cfg2")),
+        "roofline": roofline("hbm", achieved, peaks["hbm_gbs"], "GB/s", traffic.get("decode_ws:multi_stream_decode")),
         "kernels": {"decode_partial_ms": round(part_ms, 5), "merge_ms": round(per[1] / args.steps, 5)},
         "peaks_source": peaks["source"],
         "gpu_launches": 2 * args.steps,
@@ -349,7 +349,7 @@ def run_native(args):
         if want(args, "verify") or want(args, "argmax"):
             sec.update(bench_verify(wl, dev, ks, peaks, traffic))
         if want(args, "ring"):
-            sec["ring"] = bench_ring(wl, tf, dev, ks, peaks)
+            sec["ring"] = bench_ring(wl, tf, dev, ks, peaks, traffic)
         if want(args, "prompt"):
             sec["prompt"] = bench_prompt(wl, tf, dev, max(3, ks // 4), peaks)
         result["secondary"] = sec
@@ -425,19 +425,19 @@ def bench_verify(wl, dev, steps, peaks, traffic):
                    "kv_gbs": round(kv / (pms + mms) / 1e6, 2), "ms_per_step": round((pms + mms), 5),
                    "tflops": round(flops / (pms * 1e-3) / 1e12, 2),
                    "roofline": roofline("hbm", kv / (pms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                                        traffic.get("decode_partial_cfg3")),
+                                        traffic.get("attn_partial:shared_verify")),
                    "launches": 2 * steps, "l2": "8 rotating copies"},
         "argmax": {"workload": f"{rows} rows x 128,000 bf16 ~N(0,3), ties in ~1/4 of rows",
                    "rows_per_s": round(rows / (ams * 1e-3), 1), "ms": round(ams, 5),
                    "roofline": roofline("hbm", arg_bytes / (ams * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                                        traffic.get("argmax_cfg3")),
+                                        traffic.get("argmax:verify_logits")),
                    "launches": steps},
     }
     assert int(run.st.item()) == 0
     return out
 
 
-def bench_ring(wl, tf, dev, steps, peaks):
+def bench_ring(wl, tf, dev, steps, peaks, traffic):
     import torch
 
     from paged_kv_cache_segment_b200 import binding
@@ -466,7 +466,8 @@ def bench_ring(wl, tf, dev, steps, peaks):
     return {"workload": "drafter ring: 17 rows, rings of 4,200 slots, random heads, U{1000..4200} valid, 16/2 heads, "
                         "D256, 256-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
             "ms_per_step": round(ms, 5), "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
-            "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"), "launches": 2 * steps,
+            "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                                 traffic.get("decode_ws:drafter_ring")), "launches": 2 * steps,
             "l2": "3 rotating copies"}
 
 

@@ -8,8 +8,8 @@
 // key loop.
 //
 // One CTA computes 128 queries: 128/G consecutive rows x the G q-heads that
-// share kv-head g, so one K/V tile serves all of them.  Six warps split the
-// work by role: a TMA warp, an MMA warp and four softmax warps.  Per 64-key
+// share kv-head g, so one K/V tile serves all of them.  Ten warps split the
+// work by role: a TMA warp, an MMA warp and eight softmax warps.  Per 64-key
 // tile:
 //   1. the TMA warp brings K (and V) in 128-byte-swizzled 64-column slabs, one
 //      box per page (or per 64-key span of a larger page) and slab, every lane
@@ -17,9 +17,10 @@
 //      so no page-table read sits in the key loop;
 //   2. the MMA warp issues S = Q K^T (M 128, N 64, K = D) into tensor memory,
 //      one tile ahead of the softmax (two S buffers);
-//   3. every softmax thread owns one query row: it loads its S row from tensor
-//      memory, masks it causally, and folds it into a running max / sum with a
-//      lazy rescale (the reference max moves only when it rises by 2^8);
+//   3. two softmax threads share a query row, 32 key columns each: they load
+//      their S columns from tensor memory, mask them causally, swap their
+//      maxima through shared memory and fold the tile into a running max / sum
+//      with a lazy rescale (the reference max moves only when it rises by 2^8);
 //   4. the weights go back to tensor memory (into the S columns they came
 //      from) and the MMA warp issues O += P V (A from tensor memory, B = V in
 //      shared memory, MN-major).  For f32 output P is fed as bf16 hi + bf16 lo
@@ -42,8 +43,12 @@
 
 namespace tfp {
 
-constexpr int kPTSoftmax = 128;               // four softmax warps, one query row a thread
+// Eight softmax warps: warps q and q + 4 share the tensor-memory lane quadrant
+// q (query rows 32q .. 32q + 31) and take 32 of a tile's 64 key columns each,
+// so every SM sub-partition has two softmax warps to interleave.
+constexpr int kPTSoftmax = 256;
 constexpr int kPTThreads = kPTSoftmax + 64;   // + an MMA warp and a TMA warp
+constexpr int kPTMmaWarp = kPTSoftmax / 32, kPTTmaWarp = kPTMmaWarp + 1;
 constexpr int kQM = 128;                      // queries a CTA (the MMA's M)
 constexpr int kBN = 64;                       // keys a tile
 constexpr int kQSlab = kQM * 128;             // 128 query rows x 128 bytes
@@ -84,6 +89,9 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     __shared__ uint32_t s_tmem;
     __shared__ uint32_t s_vbad[4];
     __shared__ uint32_t s_err, s_abort;
+    __shared__ float s_xmax[2][2][kQM];     // [tile parity][column half][row]: the halves' tile maxima
+    __shared__ float s_xl[2][kQM];          // [column half][row]: final partial sums
+    __shared__ uint32_t s_xbad[2][2][kQM];  // [exchange][column half][row]: nonfinite findings
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -123,7 +131,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 11; ++i) mbar_init(smem_u32(&bars[i]), (i >= 7 && i <= 8) ? 4u : 1u);
+        for (int i = 0; i < 11; ++i) mbar_init(smem_u32(&bars[i]), (i >= 7 && i <= 8) ? kPTSoftmax / 32u : 1u);
         fence_barrier_init();
         s_err = 0;
         s_abort = 0;
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
 
     // every lane of a helper warp waits; the answer is the warp's, so all lanes branch alike
     auto wwait = [&](uint32_t bar, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(bar, phase, abort_flag)); };
-    if (warp == 5) {
+    if (warp == kPTTmaWarp) {
         // ================= TMA warp: the K/V boxes of a tile go out one per lane,
         // so one warp instruction issues all of them; a buffer is refilled as
         // soon as the MMA that read it is done
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             if (t >= 2 && !wwait(bo(pb), pph)) break;
             issue_kv(t, true);
         }
-    } else if (warp == 4) {
+    } else if (warp == kPTMmaWarp) {
         // ================= MMA warp: lane 0 issues every tcgen05.mma
         const uint32_t idesc_qk = umma_idesc_bf16(kQM, kBN, false, false);
         const uint32_t idesc_pv = umma_idesc_bf16(kQM, D, false, true);
@@ -230,100 +238,113 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             __syncwarp();
         }
     } else {
-        // ================= softmax warps: thread tid owns query row tid
-        const int qi = tid;
+        // ================= softmax warps: row qi of the tile, key columns 32h .. 32h + 31
+        const int quad = warp & 3, h = warp >> 2;
+        const int qi = quad * 32 + lane;
         const int row_i = row0 + qi / G;  // chunk-relative
         const bool valid_row = row_i < T;
         const int lim = valid_row ? (N - T + row_i + 1) : key_hi_eff;
         const float scale_log2 = p.scale_log2;
         float m_ref = -INFINITY, l_run = 0.f;
         uint32_t emax = 0, tail_bad = 0;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t pair_bar = 2 + quad;  // warps quad and quad + 4
 
         for (int j = 0; j < n_tiles; ++j) {
             const int b = j & 1, kt = j * kBN;
             const uint32_t ph = (uint32_t)((j >> 1) & 1);
             const uint32_t colS = b ? kColS1 : kColS0;
+            const int kh = kt + 32 * h;  // this half's first key
             pt_wait(bsq(b), ph, abort_flag);
             tc_fence_after();
-            float sv[kBN];
+            float sv[32];
             {
                 uint32_t r[32];
-                tmem_ld32(lane_base + colS, r);
+                tmem_ld32(lane_base + colS + 32 * h, r);
+                tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; ++c) sv[c] = __uint_as_float(r[c]);
-                tmem_ld32(lane_base + colS + 32, r);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) sv[32 + c] = __uint_as_float(r[c]);
             }
-            tmem_wait_ld();
-            const bool need_mask = kt + kBN > full_hi;
-            // the tile's largest score; nonfinite visible scores: NaN and +inf
-            // reach the row sum (checked at the end), -inf is caught by the min
-            float mx = -INFINITY;
-            if (need_mask) {
+            // the half's largest score (four independent chains); nonfinite
+            // visible scores: NaN and +inf reach the row sum (checked at the
+            // end), -inf is caught by the min
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (kt + kBN > full_hi) {
 #pragma unroll
-                for (int c = 0; c < kBN; ++c) {
-                    const bool vis = kt + c < lim;
+                for (int c = 0; c < 32; ++c) {
+                    const bool vis = kh + c < lim;
                     emax = max(emax, vis ? exp_bits(sv[c]) : 0u);
                     sv[c] = vis ? sv[c] : -INFINITY;
-                    mx = fmaxf(mx, sv[c]);
+                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
                 }
             } else {
-                float mn = INFINITY;
+                float n4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
 #pragma unroll
-                for (int c = 0; c < kBN; ++c) {
-                    mx = fmaxf(mx, sv[c]);
-                    mn = fminf(mn, sv[c]);
+                for (int c = 0; c < 32; ++c) {
+                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                    n4[c & 3] = fminf(n4[c & 3], sv[c]);
                 }
-                if (mn == -INFINITY) emax = 0x7f800000u;
+                if (fminf(fminf(n4[0], n4[1]), fminf(n4[2], n4[3])) == -INFINITY) emax = 0x7f800000u;
             }
+            const float mine = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // the row's tile maximum: swap halves with the partner warp
+            s_xmax[b][h][qi] = mine;
+            named_bar_sync(pair_bar, 64);
+            float mx = fmaxf(mine, s_xmax[b][h ^ 1][qi]);
             mx *= scale_log2;  // scale > 0: the max commutes with it
-            // lazy rescale: the reference max moves only when it rises by 2^8
+            // lazy rescale: the reference max moves only when it rises by 2^8;
+            // both halves see the same maximum, so they move together
             float alpha = 1.f;
             if (mx > m_ref + 8.f || (m_ref == -INFINITY && mx != -INFINITY)) {
                 alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
                 m_ref = mx;
             }
             const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+            // the weights replace the scores in tensor memory (the partner has
+            // loaded its half: it passed the pair barrier): keys 32h .. 32h + 31
+            // as bf16 pairs in columns 16h .. 16h + 15, the low parts 32 further
             {
-                uint32_t hi[32];
-                float ls = 0.f;
+                uint32_t hi[16];
+                float ls0 = 0.f, ls1 = 0.f;
                 if constexpr (HILO) {
-                    uint32_t lo[32];
+                    uint32_t lo[16];
 #pragma unroll
-                    for (int w = 0; w < 32; ++w) {
+                    for (int w = 0; w < 16; ++w) {
                         const float p0 = ex2(fmaf(sv[2 * w], scale_log2, -mu));
                         const float p1 = ex2(fmaf(sv[2 * w + 1], scale_log2, -mu));
-                        ls += p0 + p1;
+                        ls0 += p0;
+                        ls1 += p1;
                         hi[w] = pack_bf16x2(p0, p1);
                         lo[w] = pack_bf16x2(p0 - bf16_lo_to_f32(hi[w]), p1 - bf16_hi_to_f32(hi[w]));
                     }
-                    tmem_st32(lane_base + colS + 32, lo);
+                    tmem_st16(lane_base + colS + 32 + 16 * h, lo);
                 } else {
 #pragma unroll
-                    for (int w = 0; w < 32; ++w) {
+                    for (int w = 0; w < 16; ++w) {
                         const float p0 = ex2(fmaf(sv[2 * w], scale_log2, -mu));
                         const float p1 = ex2(fmaf(sv[2 * w + 1], scale_log2, -mu));
-                        ls += p0 + p1;
+                        ls0 += p0;
+                        ls1 += p1;
                         hi[w] = pack_bf16x2(p0, p1);
                     }
                 }
-                l_run = l_run * alpha + ls;
-                tmem_st32(lane_base + colS, hi);
+                l_run = l_run * alpha + (ls0 + ls1);
+                tmem_st16(lane_base + colS + 16 * h, hi);
             }
-            // O holds the tiles before this one: rescale it once P V(j-1) is done
+            // O holds the tiles before this one: rescale it once P V(j-1) is
+            // done; this half rescales O columns h * D/2 .. (h + 1) * D/2 - 1
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 pt_wait(bo((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag);
                 tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t r[32];
-                    tmem_ld32(lane_base + kColO + c * 32, r);
+                    const uint32_t col = kColO + h * (D / 2) + c * 32;
+                    tmem_ld32(lane_base + col, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int w = 0; w < 32; ++w) r[w] = __float_as_uint(__uint_as_float(r[w]) * alpha);
-                    tmem_st32(lane_base + kColO + c * 32, r);
+                    tmem_st32(lane_base + col, r);
                 }
             }
             tmem_wait_st();
@@ -376,43 +397,55 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             if (lane == 0) mbar_arrive(bpr(b));
         }
 
-        // ---- epilogue: O / l, nonfinite check, store
+        // ---- epilogue: the halves' sums and findings meet, then each half
+        // divides and stores its D/2 columns of O
         if (n_tiles > 0) pt_wait(bo((n_tiles - 1) & 1), (uint32_t)(((n_tiles - 1) >> 1) & 1), abort_flag);
         tc_fence_after();
         const bool aborted = *abort_flag != 0;
-        uint32_t bad = (emax == 0x7f800000u) | tail_bad | s_err | (aborted ? 1u : 0u);
-        if (!(l_run > 0.f) || !isfinite(l_run)) bad = 1;
+        s_xl[h][qi] = l_run;
+        s_xbad[0][h][qi] = (emax == 0x7f800000u ? 1u : 0u) | tail_bad;
+        named_bar_sync(pair_bar, 64);
+        const float l_sum = s_xl[0][qi] + s_xl[1][qi];
+        uint32_t bad = s_xbad[0][0][qi] | s_xbad[0][1][qi] | s_err | (aborted ? 1u : 0u);
+        if (!(l_sum > 0.f) || !isfinite(l_sum)) bad = 1;
         const int64_t u = (int64_t)(p.q_row + row_i) * p.hq + g * G + (qi % G);
+        const int d0 = h * (D / 2);
+        uint32_t obad = 0;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
             uint32_t r[32];
-            tmem_ld32(lane_base + kColO + c * 32, r);
+            tmem_ld32(lane_base + kColO + d0 + c * 32, r);
             tmem_wait_ld();
             float o[32];
 #pragma unroll
             for (int w = 0; w < 32; ++w) {
-                o[w] = __uint_as_float(r[w]) / l_run;
-                bad |= !isfinite(o[w]);
+                o[w] = __uint_as_float(r[w]) / l_sum;
+                obad |= !isfinite(o[w]);
             }
             if (valid_row && !aborted) {
                 if (p.out_bf16) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + c * 32);
+                    uint4 *dst =
+                        reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d0 + c * 32);
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
                         dst[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]), pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
                                             pack_bf16x2(o[8 * w + 4], o[8 * w + 5]),
                                             pack_bf16x2(o[8 * w + 6], o[8 * w + 7]));
                 } else {
-                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + c * 32);
+                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d0 + c * 32);
 #pragma unroll
                     for (int w = 0; w < 8; ++w) dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
                 }
             }
         }
+        // a nonfinite output in either half flags the whole row
+        s_xbad[1][h][qi] = obad;
+        named_bar_sync(pair_bar, 64);
+        bad |= s_xbad[1][0][qi] | s_xbad[1][1][qi];
         if (valid_row) {
             if (bad) {
                 const float qnan = __int_as_float(0x7fc00000);
-                for (int d = 0; d < D; d += 8) {
+                for (int d = d0; d < d0 + D / 2; d += 8) {
                     if (p.out_bf16)
                         *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d) =
                             make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
@@ -423,7 +456,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
                     }
                 }
             }
-            if (p.out_flags) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
+            if (p.out_flags && h == 0) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
         }
     }
     // everyone: report a timeout, give in-flight work a bounded chance to land,
