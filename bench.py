@@ -424,8 +424,9 @@ def bench_verify(wl, dev, steps, peaks, traffic):
                                "U{2048..16384}, 1024-key partials + merge", "rows": rows,
                    "kv_gbs": round(kv / (pms + mms) / 1e6, 2), "ms_per_step": round((pms + mms), 5),
                    "tflops": round(flops / (pms * 1e-3) / 1e12, 2),
-                   "roofline": roofline("hbm", kv / (pms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
-                                        traffic.get("attn_partial:shared_verify")),
+                   "roofline": dict(roofline("hbm", kv / (pms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                                             traffic.get("prompt_tc:shared_verify")),
+                                    kernel="prompt_tc_kernel<256, hilo, partial>"),
                    "launches": 2 * steps, "l2": "8 rotating copies"},
         "argmax": {"workload": f"{rows} rows x 128,000 bf16 ~N(0,3), ties in ~1/4 of rows",
                    "rows_per_s": round(rows / (ams * 1e-3), 1), "ms": round(ams, 5),

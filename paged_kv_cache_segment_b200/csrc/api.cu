@@ -149,6 +149,37 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
             launch_decode_ws(w, head_dim, false, k_pool, v_pool, items, reinterpret_cast<cudaStream_t>(stream)));
     }
 
+    // more queries per kv-head (a verify round): the tcgen05 kernel, one CTA
+    // per (stream, kv-head, split, 128-query tile)
+    if (partial_tc_supported(head_dim, group, page_size, split_keys)) {
+        const int rt = 128 / group;
+        const int64_t n_qt = ((int64_t)max_rows + rt - 1) / rt;
+        if (n_qt * n_splits_max <= 0x7fffffff) {
+            PromptTcParams t{};
+            t.q = static_cast<const uint16_t *>(q);
+            t.page_table = page_table;
+            t.n_pages = n_pages;
+            t.log2_page = lp;
+            t.hq = n_q_heads;
+            t.hkv = n_kv_heads;
+            t.group = group;
+            t.n_rows_total = n_rows_total;
+            t.scale_log2 = scale * 1.4426950408889634f;
+            t.segs = segs;
+            t.pt_len = page_table_len;
+            t.split_keys = split_keys;
+            t.n_splits_max = n_splits_max;
+            t.n_qt = (int)n_qt;
+            t.part_o = part_o;
+            t.part_m = part_m;
+            t.part_l = part_l;
+            t.part_flag = part_flag;
+            t.status = status;
+            return cuda_status(
+                launch_partial_tc(t, head_dim, k_pool, v_pool, n_segs, reinterpret_cast<cudaStream_t>(stream)));
+        }
+    }
+
     AttnParams p{};
     p.q = static_cast<const uint16_t *>(q);
     p.n_rows_total = n_rows_total;
@@ -222,6 +253,7 @@ tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_
 
     if (prompt_tc_supported(head_dim, group, page_size)) {
         PromptTcParams t{};
+        t.q = static_cast<const uint16_t *>(q);
         t.q_row = seg_host->q_row;
         t.n_rows = seg_host->n_rows;
         t.n_keys = seg_host->n_keys;
@@ -239,7 +271,7 @@ tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_
         t.out_bf16 = out_dtype == TF_OUT_BF16;
         t.out_flags = flags;
         t.status = status;
-        return cuda_status(launch_prompt_tc(t, head_dim, q, k_pool, v_pool, reinterpret_cast<cudaStream_t>(stream)));
+        return cuda_status(launch_prompt_tc(t, head_dim, k_pool, v_pool, reinterpret_cast<cudaStream_t>(stream)));
     }
     AttnParams p{};
     p.q = static_cast<const uint16_t *>(q);

@@ -17,7 +17,9 @@
 // among the words it still holds in registers (an IEEE compare, so -0 equals
 // +0), and the CTAs' first columns meet on rank 0 the same way.  No
 // workspace and no inter-CTA counters: the cluster barriers order the
-// exchanges.
+// exchanges, and a first split barrier (arrive at entry, wait before the
+// first remote store) makes sure every CTA of the cluster has started before
+// any of them writes into another's shared memory.
 
 #include <cooperative_groups.h>
 
@@ -68,6 +70,11 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
     const int per = ((p.n_cols + kArgmaxCluster * 8 - 1) / (kArgmaxCluster * 8)) * 8;
     const int c0 = min(p.n_cols, rank * per), c1 = min(p.n_cols, c0 + per);
     const uint32_t kNegInf2 = 0xff80ff80u, kPad2 = 0xff7fff7fu;
+    // A CTA may touch another CTA's shared memory only once every CTA of the
+    // cluster is running: arrive here, wait before the first remote store
+    // (the loads of pass 1 overlap the wait).
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    bool joined = false;
 
     for (int row = blockIdx.y; row < p.n_rows; row += gridDim.y) {
         const uint16_t *rp = p.logits + (int64_t)row * p.ld;
@@ -118,6 +125,10 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
         k = __reduce_max_sync(0xffffffffu, k);
         const uint32_t wbad = __reduce_or_sync(0xffffffffu, bad);
         if (lane == 0) w_red[warp] = k | (wbad << 31);
+        if (!joined) {
+            asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+            joined = true;
+        }
         __syncthreads();
         if (tid < kArgmaxCluster) {
             uint32_t m = 0;

@@ -16,7 +16,10 @@
 //      issuing one box; the CTA's page ids were copied to shared memory once,
 //      so no page-table read sits in the key loop;
 //   2. the MMA warp issues S = Q K^T (M 128, N 64, K = D) into tensor memory,
-//      one tile ahead of the softmax (two S buffers);
+//      one tile ahead of the softmax (two S buffers).  Q itself sits in tensor
+//      memory (the softmax warps put it there once), so the MMAs read only K
+//      from shared memory: shared-memory bandwidth, not the tensor pipe, is
+//      what an M = 128 tile runs out of first;
 //   3. two softmax threads share a query row, 32 key columns each: they load
 //      their S columns from tensor memory, mask them causally, swap their
 //      maxima through shared memory and fold the tile into a running max / sum
@@ -27,8 +30,8 @@
 //      (two MMAs, about 16 bits a weight, so the fp32 tolerance holds); for
 //      bf16 output P is one bf16, whose rounding is below the output's own;
 //   5. O stays in tensor memory until the epilogue divides by the sum.
-// K and V each have two buffers; a buffer is refilled as soon as the MMA that
-// read it has completed.
+// K and V each have three buffers; a buffer is refilled as soon as the MMA
+// that read it has completed.
 // Nonfinite handling matches the other attention kernels: visible scores are
 // checked through their exponent bits, value rows that only some rows see
 // are scanned and zeroed, and the final O and sum are checked.
@@ -51,20 +54,20 @@ constexpr int kPTThreads = kPTSoftmax + 64;   // + an MMA warp and a TMA warp
 constexpr int kPTMmaWarp = kPTSoftmax / 32, kPTTmaWarp = kPTMmaWarp + 1;
 constexpr int kQM = 128;                      // queries a CTA (the MMA's M)
 constexpr int kBN = 64;                       // keys a tile
-constexpr int kQSlab = kQM * 128;             // 128 query rows x 128 bytes
 constexpr int kKVSlab = kBN * 128;            // 64 key rows x 128 bytes
-constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 256;  // tensor-memory columns
+constexpr int kKVStages = 3;                  // K and V buffers in flight
+// tensor-memory columns: two S tiles, Q (D/2 columns of bf16 pairs), O
+constexpr uint32_t kColS0 = 0, kColS1 = 64, kColQ = 128, kColO = 256;
 
 template <int D>
 struct PTCfg {
     static constexpr int kSlabs = D / 64;
-    static constexpr int kQBytes = kSlabs * kQSlab;
     static constexpr int kKVBytes = kSlabs * kKVSlab;
-    // Q, two K buffers, two V buffers
-    static constexpr int kOffK = kQBytes;
-    static constexpr int kOffV = kQBytes + 2 * kKVBytes;
+    // kKVStages K buffers, then kKVStages V buffers, then the page ids
+    static constexpr int kOffK = 0;
+    static constexpr int kOffV = kKVStages * kKVBytes;
     static constexpr int kPidCap = 4096;  // page ids held in shared memory (16 KB)
-    static constexpr int kOffPid = kQBytes + 4 * kKVBytes;
+    static constexpr int kOffPid = 2 * kKVStages * kKVBytes;
     static constexpr int kSmemBytes = kOffPid + kPidCap * 4 + 1024;
     static constexpr uint32_t kTmemCols = 512;
 };
@@ -78,14 +81,24 @@ __device__ __forceinline__ bool pt_wait(uint32_t bar, uint32_t phase, volatile u
     return false;
 }
 
-template <int D, bool HILO>
+// barrier slots
+constexpr int kBarQ = 0;                            // Q in tensor memory (softmax warps arrive)
+constexpr int kBarKFull = 1;                        // [kKVStages] K tile landed
+constexpr int kBarVFull = kBarKFull + kKVStages;    // [kKVStages] V tile landed
+constexpr int kBarKFree = kBarVFull + kKVStages;    // [kKVStages] QK that read the K buffer done
+constexpr int kBarVFree = kBarKFree + kKVStages;    // [kKVStages] P V that read the V buffer done
+constexpr int kBarS = kBarVFree + kKVStages;        // [2] QK done: S tile ready
+constexpr int kBarPr = kBarS + 2;                   // [2] P written, V cleaned (softmax warps arrive)
+constexpr int kBarO = kBarPr + 2;                   // [2] P V done
+constexpr int kNumBars = kBarO + 2;
+
+template <int D, bool HILO, bool PARTIAL>
 __global__ void __launch_bounds__(kPTThreads, 1)
-    prompt_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const PromptTcParams p) {
+    prompt_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const PromptTcParams p) {
     using C = PTCfg<D>;
     extern __shared__ unsigned char smem_raw[];
-    // barriers: q; k[2]; v[2]; s[2] (QK done); pr[2] (P written, V cleaned); o[2] (PV done)
-    __shared__ __align__(8) uint64_t bars[11];
+    __shared__ __align__(8) uint64_t bars[kNumBars];
     __shared__ uint32_t s_tmem;
     __shared__ uint32_t s_vbad[4];
     __shared__ uint32_t s_err, s_abort;
@@ -96,34 +109,85 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *sbase_ptr = smem_raw + (sbase - smem_u32(smem_raw));
-    const uint32_t sQ = sbase;
-    auto sK = [&](int b) { return sbase + C::kOffK + b * C::kKVBytes; };
-    auto sV = [&](int b) { return sbase + C::kOffV + b * C::kKVBytes; };
-    const uint32_t bq = smem_u32(&bars[0]);
-    auto bk = [&](int b) { return smem_u32(&bars[1 + b]); };
-    auto bv = [&](int b) { return smem_u32(&bars[3 + b]); };
-    auto bsq = [&](int b) { return smem_u32(&bars[5 + b]); };
-    auto bpr = [&](int b) { return smem_u32(&bars[7 + b]); };
-    auto bo = [&](int b) { return smem_u32(&bars[9 + b]); };
+    auto sK = [&](int s) { return sbase + C::kOffK + s * C::kKVBytes; };
+    auto sV = [&](int s) { return sbase + C::kOffV + s * C::kKVBytes; };
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
     volatile uint32_t *abort_flag = &s_abort;
 
     const int G = p.group, RT = kQM / p.group;  // rows a tile
     const int g = blockIdx.y;
-    const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;  // the most keys first
-    const int row0 = qt * RT;                              // chunk-relative first row
-    const int T = p.n_rows, N = p.n_keys;
-    const int rows_here = min(RT, T - row0);
-    const int key_hi_eff = N - T + row0 + rows_here;  // keys the last valid row sees
-    const int full_hi = N - T + row0 + 1;             // keys every row of the tile sees
-    const int n_tiles = (key_hi_eff + kBN - 1) / kBN;
     const int P = 1 << p.log2_page, BR = P < kBN ? P : kBN, n_box = kBN / BR;
 
-    // The CTA's page ids, read once here by every thread (coalesced), so the
-    // issuer never waits on a page-table read inside the key loop.
+    // ---- the work item: a segment (the prompt's one, or entry blockIdx.z of
+    // the table), a tile of 128/G rows and, for partials, a split of the keys
+    int q_row = p.q_row, T = p.n_rows, N = p.n_keys, pt_base = p.pt_base, n_pg = p.n_pg;
+    int qt, split = 0, key_lo = 0, key_hi_split;
+    if constexpr (PARTIAL) {
+        const tf_seg sg = p.segs[blockIdx.z];
+        q_row = sg.q_row;
+        T = sg.n_rows;
+        N = sg.n_keys;
+        pt_base = sg.pt_base;
+        n_pg = sg.n_pages;
+        split = (int)blockIdx.x / p.n_qt;
+        qt = p.n_qt - 1 - (int)blockIdx.x % p.n_qt;  // the most keys first
+        const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < T || pt_base < 0 ||
+                         n_pg < 0 || (int64_t)pt_base + n_pg > p.pt_len;
+        if (bad) {
+            if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
+            return;
+        }
+        if ((int64_t)N > ((int64_t)n_pg << p.log2_page)) {
+            if (tid == 0) atomicOr(p.status, TF_DEV_PAST_PAGES);
+            return;
+        }
+        const int n_sp = (N + p.split_keys - 1) / p.split_keys;
+        if (n_sp > p.n_splits_max) {
+            if (tid == 0) atomicOr(p.status, TF_DEV_SPLITS);
+            return;
+        }
+        if (qt * RT >= T) return;
+        if (split >= n_sp) {
+            // a partial slot past the stream's count: an empty partial, o untouched
+            for (int r = tid; r < min(RT, T - qt * RT) * G; r += kPTThreads) {
+                const int64_t at = ((int64_t)(q_row + qt * RT + r / G) * p.hq + g * G + r % G) * p.n_splits_max + split;
+                p.part_m[at] = -INFINITY;
+                p.part_l[at] = 0.f;
+                p.part_flag[at] = 0;
+            }
+            return;
+        }
+        key_lo = split * p.split_keys;
+        key_hi_split = min(N, key_lo + p.split_keys);
+    } else {
+        qt = (int)gridDim.x - 1 - (int)blockIdx.x;  // the most keys first
+        key_hi_split = N;
+    }
+    const int row0 = qt * RT;  // segment-relative first row
+    const int rows_here = min(RT, T - row0);
+    const int key_hi_eff = min(key_hi_split, N - T + row0 + rows_here);  // keys the last valid row sees
+    const int full_hi = min(key_hi_eff, N - T + row0 + 1);               // keys every row of the tile sees
+    const int n_tiles = key_hi_eff > key_lo ? (key_hi_eff - key_lo + kBN - 1) / kBN : 0;
+    if (PARTIAL && n_tiles == 0) {
+        // no row of the tile sees a key of this split: m = -inf, l = 0, o = 0
+        for (int r = tid; r < rows_here * G; r += kPTThreads) {
+            const int64_t at = ((int64_t)(q_row + row0 + r / G) * p.hq + g * G + r % G) * p.n_splits_max + split;
+            p.part_m[at] = -INFINITY;
+            p.part_l[at] = 0.f;
+            p.part_flag[at] = 0;
+            for (int d = 0; d < D; d += 4) *reinterpret_cast<float4 *>(p.part_o + at * D + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+
+    // The CTA's page ids (pages pg_lo .. of its key range), read once here by
+    // every thread (coalesced), so the TMA warp never waits on a page-table
+    // read inside the key loop.
     int *pids = reinterpret_cast<int *>(sbase_ptr + C::kOffPid);
-    const int n_pid = min((key_hi_eff + P - 1) >> p.log2_page, p.n_pg);
+    const int pg_lo = key_lo >> p.log2_page;
+    const int n_pid = min((key_hi_eff + P - 1) >> p.log2_page, n_pg) - pg_lo;
     for (int i = tid; i < n_pid && i < C::kPidCap; i += kPTThreads) {
-        const int id = p.page_table[p.pt_base + i];
+        const int id = p.page_table[pt_base + pg_lo + i];
         pids[i] = (id < 0 || id >= p.n_pages) ? -1 : id;
     }
     if (warp == 0) {
@@ -131,7 +195,8 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 11; ++i) mbar_init(smem_u32(&bars[i]), (i >= 7 && i <= 8) ? kPTSoftmax / 32u : 1u);
+        for (int i = 0; i < kNumBars; ++i)
+            mbar_init(bar(i), (i == kBarQ || i == kBarPr || i == kBarPr + 1) ? kPTSoftmax / 32u : 1u);
         fence_barrier_init();
         s_err = 0;
         s_abort = 0;
@@ -143,23 +208,23 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     const uint32_t tmem = s_tmem;
 
     // every lane of a helper warp waits; the answer is the warp's, so all lanes branch alike
-    auto wwait = [&](uint32_t bar, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(bar, phase, abort_flag)); };
+    auto wwait = [&](uint32_t b, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(b, phase, abort_flag)); };
     if (warp == kPTTmaWarp) {
         // ================= TMA warp: the K/V boxes of a tile go out one per lane,
         // so one warp instruction issues all of them; a buffer is refilled as
         // soon as the MMA that read it is done
         if (lane == 0) {
-            prefetch_tensormap(&tmQ);
             prefetch_tensormap(&tmK);
             prefetch_tensormap(&tmV);
         }
         const int n_copies = n_box * C::kSlabs;  // boxes of one K (or V) tile, <= 32
-        // K or V tile t into buffer t & 1: one box per page (or per 64-key span
-        // of a larger page) and 64-column slab; page ids come from shared memory
+        // K or V tile t into stage t % kKVStages: one box per page (or per
+        // 64-key span of a larger page) and 64-column slab; page ids come from
+        // shared memory
         auto issue_kv = [&](int t, bool is_v) {
-            const int kt = t * kBN, b = t & 1;
-            const uint32_t dst0 = is_v ? sV(b) : sK(b);
-            const uint32_t bar = is_v ? bv(b) : bk(b);
+            const int kt = key_lo + t * kBN, s = t % kKVStages;
+            const uint32_t dst0 = is_v ? sV(s) : sK(s);
+            const uint32_t full = bar((is_v ? kBarVFull : kBarKFull) + s);
             const CUtensorMap *map = is_v ? &tmV : &tmK;
             // lane i < n_copies owns box x = i / slabs, slab sl = i % slabs
             const int x = lane / C::kSlabs, sl = lane % C::kSlabs;
@@ -167,12 +232,12 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             int id = -1;
             if (lane < n_copies && key0 < key_hi_eff) {
                 const int idx = key0 >> p.log2_page;
-                if (idx >= p.n_pg)
+                if (idx >= n_pg)
                     id = -2;
-                else if (idx < C::kPidCap)
-                    id = pids[idx];
+                else if (idx - pg_lo < C::kPidCap)
+                    id = pids[idx - pg_lo];
                 else  // past the shared-memory copy (very long prompts with small pages)
-                    id = p.page_table[p.pt_base + idx];
+                    id = p.page_table[pt_base + idx];
                 if (id < 0 || id >= p.n_pages) {
                     id = -1;
                     s_err = 1;
@@ -180,60 +245,60 @@ __global__ void __launch_bounds__(kPTThreads, 1)
                 }
             }
             const uint32_t live = __ballot_sync(0xffffffffu, id >= 0);
-            if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)__popc(live) * (uint32_t)(BR * 128));
+            if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)__popc(live) * (uint32_t)(BR * 128));
             __syncwarp();
-            if (id >= 0) tma_load_4d(dst0 + sl * kKVSlab + x * BR * 128, map, bar, 64 * sl, key0 & (P - 1), g, id);
+            if (id >= 0) tma_load_4d(dst0 + sl * kKVSlab + x * BR * 128, map, full, 64 * sl, key0 & (P - 1), g, id);
         };
-        if (lane == 0) mbar_arrive_expect_tx(bq, (uint32_t)C::kQBytes);
-        __syncwarp();
-        if (lane < C::kSlabs) tma_load_3d(sQ + lane * kQSlab, &tmQ, bq, 64 * lane, g * G, p.q_row + row0);
         for (int t = 0; t < n_tiles; ++t) {
-            const int pb = (t - 2) & 1;
-            const uint32_t pph = (uint32_t)(((t - 2) >> 1) & 1);
-            // K(t) once QK(t-2) has read the buffer, V(t) once P V(t-2) has
-            if (t >= 2 && !wwait(bsq(pb), pph)) break;
+            const int s = t % kKVStages;
+            const uint32_t fph = (uint32_t)((t / kKVStages - 1) & 1);  // completion of tile t - kKVStages
+            // K(t) once QK(t - stages) has read the buffer, V(t) once P V(t - stages) has
+            if (t >= kKVStages && !wwait(bar(kBarKFree + s), fph)) break;
             issue_kv(t, false);
-            if (t >= 2 && !wwait(bo(pb), pph)) break;
+            if (t >= kKVStages && !wwait(bar(kBarVFree + s), fph)) break;
             issue_kv(t, true);
         }
     } else if (warp == kPTMmaWarp) {
         // ================= MMA warp: lane 0 issues every tcgen05.mma
         const uint32_t idesc_qk = umma_idesc_bf16(kQM, kBN, false, false);
         const uint32_t idesc_pv = umma_idesc_bf16(kQM, D, false, true);
+        // S(t) = Q K(t)^T with Q (the A operand) in tensor memory
         auto issue_qk = [&](int t) {
             if (lane == 0) {
-                const int b = t & 1;
+                const int b = t & 1, s = t % kKVStages;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const int sl = k >> 2, kk = k & 3;
-                    const uint64_t ad = umma_desc_sw128(sQ + sl * kQSlab + kk * 32, 16, 1024);
-                    const uint64_t bd = umma_desc_sw128(sK(b) + sl * kKVSlab + kk * 32, 16, 1024);
-                    umma_ss(tmem + (b ? kColS1 : kColS0), ad, bd, idesc_qk, k > 0 ? 1u : 0u);
+                    const uint64_t bd = umma_desc_sw128(sK(s) + sl * kKVSlab + kk * 32, 16, 1024);
+                    umma_ts(tmem + (b ? kColS1 : kColS0), tmem + kColQ + k * 8, bd, idesc_qk, k > 0 ? 1u : 0u);
                 }
-                umma_commit(bsq(b));
+                umma_commit(bar(kBarS + b));
+                umma_commit(bar(kBarKFree + s));
             }
             __syncwarp();
         };
-        if (n_tiles > 0 && wwait(bq, 0) && wwait(bk(0), 0)) issue_qk(0);
+        if (n_tiles > 0 && wwait(bar(kBarQ), 0) && wwait(bar(kBarKFull), 0)) issue_qk(0);
         for (int j = 0; j < n_tiles; ++j) {
-            const int b = j & 1;
-            const uint32_t ph = (uint32_t)((j >> 1) & 1);
+            const int b = j & 1, s = j % kKVStages;
             // the next tile's scores while the softmax warps work on this one;
             // its S buffer held P(j-1), whose P V was issued before (in order)
-            if (j + 1 < n_tiles && wwait(bk((j + 1) & 1), (uint32_t)(((j + 1) >> 1) & 1))) issue_qk(j + 1);
+            const int j1 = j + 1;
+            if (j1 < n_tiles && wwait(bar(kBarKFull + j1 % kKVStages), (uint32_t)((j1 / kKVStages) & 1))) issue_qk(j1);
             // P(j) written (and V(j) cleaned) and V(j) landed: O += P V
-            const bool ok = wwait(bpr(b), ph) && wwait(bv(b), ph);
+            const bool ok = wwait(bar(kBarPr + b), (uint32_t)((j >> 1) & 1)) &&
+                            wwait(bar(kBarVFull + s), (uint32_t)((j / kKVStages) & 1));
             if (ok && lane == 0) {
                 tc_fence_after();
                 const uint32_t sb = tmem + (b ? kColS1 : kColS0);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t bd = umma_desc_sw128(sV(b) + kk * 16 * 128, kKVSlab, 1024);
+                    const uint64_t bd = umma_desc_sw128(sV(s) + kk * 16 * 128, kKVSlab, 1024);
                     umma_ts(tmem + kColO, sb + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                     if (HILO) umma_ts(tmem + kColO, sb + 32 + kk * 8, bd, idesc_pv, 1u);
                 }
-                umma_commit(bo(b));
+                umma_commit(bar(kBarO + b));
+                umma_commit(bar(kBarVFree + s));
             }
             __syncwarp();
         }
@@ -250,12 +315,36 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t pair_bar = 2 + quad;  // warps quad and quad + 4
 
+        // Q into tensor memory, the A operand of every QK: this thread's half
+        // of its row straight from global memory (bf16 pairs are the operand's
+        // 32-bit columns as they are); rows past the chunk are zero
+        {
+            constexpr int kWH = D / 4;  // 32-bit words a half row
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.q + ((int64_t)(q_row + (valid_row ? row_i : 0)) * p.hq + g * G + qi % G) * D + h * (D / 2));
+            uint32_t w[kWH / 16][16];
+#pragma unroll
+            for (int v = 0; v < kWH / 4; ++v) {
+                const uint4 x = valid_row ? __ldg(src + v) : make_uint4(0u, 0u, 0u, 0u);
+                w[v >> 2][4 * (v & 3)] = x.x;
+                w[v >> 2][4 * (v & 3) + 1] = x.y;
+                w[v >> 2][4 * (v & 3) + 2] = x.z;
+                w[v >> 2][4 * (v & 3) + 3] = x.w;
+            }
+#pragma unroll
+            for (int c = 0; c < kWH / 16; ++c) tmem_st16(lane_base + kColQ + h * kWH + c * 16, w[c]);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarQ));
+        }
+
         for (int j = 0; j < n_tiles; ++j) {
-            const int b = j & 1, kt = j * kBN;
+            const int b = j & 1, kt = key_lo + j * kBN;
             const uint32_t ph = (uint32_t)((j >> 1) & 1);
             const uint32_t colS = b ? kColS1 : kColS0;
             const int kh = kt + 32 * h;  // this half's first key
-            pt_wait(bsq(b), ph, abort_flag);
+            pt_wait(bar(kBarS + b), ph, abort_flag);
             tc_fence_after();
             float sv[32];
             {
@@ -334,7 +423,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             // O holds the tiles before this one: rescale it once P V(j-1) is
             // done; this half rescales O columns h * D/2 .. (h + 1) * D/2 - 1
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                pt_wait(bo((j - 1) & 1), (uint32_t)(((j - 1) >> 1) & 1), abort_flag);
+                pt_wait(bar(kBarO + ((j - 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1), abort_flag);
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < D / 64; ++c) {
@@ -351,11 +440,11 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             // V rows this tile must not feed into P V: past every row's keys ->
             // zero; seen by only some rows and nonfinite -> zero and flag
             if (kt + kBN > full_hi) {
-                pt_wait(bv(b), ph, abort_flag);
+                pt_wait(bar(kBarVFull + j % kKVStages), (uint32_t)((j / kKVStages) & 1), abort_flag);
                 named_bar_sync(1, kPTSoftmax);
                 if (tid == 0) s_vbad[0] = s_vbad[1] = 0;
                 named_bar_sync(1, kPTSoftmax);
-                unsigned char *vb = sbase_ptr + C::kOffV + b * C::kKVBytes;
+                unsigned char *vb = sbase_ptr + C::kOffV + (j % kKVStages) * C::kKVBytes;
                 for (int idx = tid; idx < kBN * C::kSlabs; idx += kPTSoftmax) {
                     const int r = idx % kBN, sl = idx / kBN;
                     uint4 *rowp = reinterpret_cast<uint4 *>(vb + sl * kKVSlab + r * 128);
@@ -394,12 +483,12 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bpr(b));
+            if (lane == 0) mbar_arrive(bar(kBarPr + b));
         }
 
         // ---- epilogue: the halves' sums and findings meet, then each half
-        // divides and stores its D/2 columns of O
-        if (n_tiles > 0) pt_wait(bo((n_tiles - 1) & 1), (uint32_t)(((n_tiles - 1) >> 1) & 1), abort_flag);
+        // stores its D/2 columns of O (divided by the sum, or raw for a partial)
+        if (n_tiles > 0) pt_wait(bar(kBarO + ((n_tiles - 1) & 1)), (uint32_t)(((n_tiles - 1) >> 1) & 1), abort_flag);
         tc_fence_after();
         const bool aborted = *abort_flag != 0;
         s_xl[h][qi] = l_run;
@@ -407,32 +496,38 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         named_bar_sync(pair_bar, 64);
         const float l_sum = s_xl[0][qi] + s_xl[1][qi];
         uint32_t bad = s_xbad[0][0][qi] | s_xbad[0][1][qi] | s_err | (aborted ? 1u : 0u);
-        if (!(l_sum > 0.f) || !isfinite(l_sum)) bad = 1;
-        const int64_t u = (int64_t)(p.q_row + row_i) * p.hq + g * G + (qi % G);
+        // a finished row always sees a key; a partial row may see none here
+        if (!isfinite(l_sum) || (!PARTIAL && !(l_sum > 0.f))) bad = 1;
+        const int64_t u = (int64_t)(q_row + row_i) * p.hq + g * G + (qi % G);
+        const int64_t at = u * (PARTIAL ? p.n_splits_max : 1) + split;  // partial slot
         const int d0 = h * (D / 2);
         uint32_t obad = 0;
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
+        for (int cc = 0; cc < D / 64; ++cc) {
             uint32_t r[32];
-            tmem_ld32(lane_base + kColO + d0 + c * 32, r);
+            tmem_ld32(lane_base + kColO + d0 + cc * 32, r);
             tmem_wait_ld();
             float o[32];
 #pragma unroll
             for (int w = 0; w < 32; ++w) {
-                o[w] = __uint_as_float(r[w]) / l_sum;
+                o[w] = PARTIAL ? __uint_as_float(r[w]) : __uint_as_float(r[w]) / l_sum;
                 obad |= !isfinite(o[w]);
             }
             if (valid_row && !aborted) {
-                if (p.out_bf16) {
+                if (PARTIAL) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.part_o + at * D + d0 + cc * 32);
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
+                } else if (p.out_bf16) {
                     uint4 *dst =
-                        reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d0 + c * 32);
+                        reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d0 + cc * 32);
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
                         dst[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]), pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
                                             pack_bf16x2(o[8 * w + 4], o[8 * w + 5]),
                                             pack_bf16x2(o[8 * w + 6], o[8 * w + 7]));
                 } else {
-                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d0 + c * 32);
+                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d0 + cc * 32);
 #pragma unroll
                     for (int w = 0; w < 8; ++w) dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
                 }
@@ -443,20 +538,30 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         named_bar_sync(pair_bar, 64);
         bad |= s_xbad[1][0][qi] | s_xbad[1][1][qi];
         if (valid_row) {
-            if (bad) {
-                const float qnan = __int_as_float(0x7fc00000);
-                for (int d = d0; d < d0 + D / 2; d += 8) {
-                    if (p.out_bf16)
-                        *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d) =
-                            make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
-                    else {
-                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d);
-                        dst[0] = make_float4(qnan, qnan, qnan, qnan);
-                        dst[1] = make_float4(qnan, qnan, qnan, qnan);
+            if (PARTIAL) {
+                // natural-log reference max, sum, flag: the merge weighs partial
+                // c by e^(m_c - M); a flagged partial flags the merged head
+                if (h == 0) {
+                    p.part_m[at] = (m_ref == -INFINITY) ? -INFINITY : m_ref * kLn2;
+                    p.part_l[at] = l_sum;
+                    p.part_flag[at] = (uint8_t)(bad ? 1 : 0);
+                }
+            } else {
+                if (bad) {
+                    const float qnan = __int_as_float(0x7fc00000);
+                    for (int d = d0; d < d0 + D / 2; d += 8) {
+                        if (p.out_bf16)
+                            *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d) =
+                                make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
+                        else {
+                            float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d);
+                            dst[0] = make_float4(qnan, qnan, qnan, qnan);
+                            dst[1] = make_float4(qnan, qnan, qnan, qnan);
+                        }
                     }
                 }
+                if (p.out_flags && h == 0) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
             }
-            if (p.out_flags && h == 0) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
         }
     }
     // everyone: report a timeout, give in-flight work a bounded chance to land,
@@ -465,9 +570,9 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     if (s_abort) {
         if (tid == 0) atomicOr(p.status, TF_DEV_TIMEOUT);
         if (tid == 0)
-            for (int i = 0; i < 11; ++i) {
-                mbar_wait(smem_u32(&bars[i]), 0u, 20000000ull);
-                mbar_wait(smem_u32(&bars[i]), 1u, 20000000ull);
+            for (int i = 0; i < kNumBars; ++i) {
+                mbar_wait(bar(i), 0u, 20000000ull);
+                mbar_wait(bar(i), 1u, 20000000ull);
             }
         __syncthreads();
     }
@@ -488,17 +593,10 @@ bool prompt_tc_supported(int head_dim, int group, int page_size) {
            (128 % group) == 0 && page_size >= 8;
 }
 
-template <int D>
-static cudaError_t launch_prompt_tc_t(const PromptTcParams &p, const void *q, const void *k, const void *v,
-                                      cudaStream_t st) {
-    CUtensorMap mq, mk, mv;
-    const int G = p.group, RT = kQM / G, P = 1 << p.log2_page, BR = P < kBN ? P : kBN;
-    {
-        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.hq, (cuuint64_t)p.n_rows_total};
-        const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.hq * D * 2};
-        const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)RT};
-        if (!make_tensor_map_bf16(&mq, q, 3, dims, strides, box)) return cudaErrorInvalidValue;
-    }
+template <int D, bool PARTIAL>
+static cudaError_t launch_tc_t(const PromptTcParams &p, const void *k, const void *v, int n_segs, cudaStream_t st) {
+    CUtensorMap mk, mv;
+    const int RT = kQM / p.group, P = 1 << p.log2_page, BR = P < kBN ? P : kBN;
     {
         const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)p.hkv, (cuuint64_t)p.n_pages};
         const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)P * D * 2, (cuuint64_t)p.hkv * P * D * 2};
@@ -506,20 +604,37 @@ static cudaError_t launch_prompt_tc_t(const PromptTcParams &p, const void *q, co
         if (!make_tensor_map_bf16(&mk, k, 4, dims, strides, box)) return cudaErrorInvalidValue;
         if (!make_tensor_map_bf16(&mv, v, 4, dims, strides, box)) return cudaErrorInvalidValue;
     }
-    auto kern = p.out_bf16 ? prompt_tc_kernel<D, false> : prompt_tc_kernel<D, true>;
+    // partials are fp32: P goes in as bf16 hi + lo
+    auto kern = PARTIAL ? prompt_tc_kernel<D, true, true>
+                        : (p.out_bf16 ? prompt_tc_kernel<D, false, false> : prompt_tc_kernel<D, true, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PTCfg<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)((p.n_rows + RT - 1) / RT), (unsigned)p.hkv);
-    kern<<<grid, kPTThreads, PTCfg<D>::kSmemBytes, st>>>(mq, mk, mv, p);
+    const dim3 grid = PARTIAL ? dim3((unsigned)(p.n_qt * p.n_splits_max), (unsigned)p.hkv, (unsigned)n_segs)
+                              : dim3((unsigned)((p.n_rows + RT - 1) / RT), (unsigned)p.hkv);
+    kern<<<grid, kPTThreads, PTCfg<D>::kSmemBytes, st>>>(mk, mv, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *q, const void *k, const void *v,
-                             cudaStream_t st) {
+cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, cudaStream_t st) {
     switch (head_dim) {
-        case 64: return launch_prompt_tc_t<64>(p, q, k, v, st);
-        case 128: return launch_prompt_tc_t<128>(p, q, k, v, st);
-        case 256: return launch_prompt_tc_t<256>(p, q, k, v, st);
+        case 64: return launch_tc_t<64, false>(p, k, v, 1, st);
+        case 128: return launch_tc_t<128, false>(p, k, v, 1, st);
+        case 256: return launch_tc_t<256, false>(p, k, v, 1, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+bool partial_tc_supported(int head_dim, int group, int page_size, int split_keys) {
+    return prompt_tc_supported(head_dim, group, page_size) && split_keys > 0 && split_keys % kBN == 0;
+}
+
+cudaError_t launch_partial_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, int n_segs,
+                              cudaStream_t st) {
+    if (n_segs == 0) return cudaSuccess;
+    switch (head_dim) {
+        case 64: return launch_tc_t<64, true>(p, k, v, n_segs, st);
+        case 128: return launch_tc_t<128, true>(p, k, v, n_segs, st);
+        case 256: return launch_tc_t<256, true>(p, k, v, n_segs, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -49,13 +49,20 @@ struct MergeParams {
 
 // Parameters of the tensor-core prompt kernel (one stream's chunk).
 struct PromptTcParams {
-    int q_row, n_rows, n_keys, pt_base, n_pg;  // the chunk's segment
+    const uint16_t *q;                         // bf16 [n_rows_total][hq][D]
+    int q_row, n_rows, n_keys, pt_base, n_pg;  // the prompt chunk's segment
     const int32_t *page_table;
     int n_pages, log2_page, hq, hkv, group, n_rows_total;
     float scale_log2;
+    // prompt: final rows
     void *out;
     int out_bf16;
     uint8_t *out_flags;
+    // split-KV partials: segment table, splits, q-tiles of the grid, outputs
+    const tf_seg *segs;
+    int pt_len, split_keys, n_splits_max, n_qt;
+    float *part_o, *part_m, *part_l;
+    uint8_t *part_flag;
     uint32_t *status;
 };
 
@@ -94,8 +101,10 @@ bool prompt_tc_supported(int head_dim, int group, int page_size);
 bool decode_ws_supported(int head_dim, int n_segs);
 cudaError_t launch_decode_ws(const WsParams &p, int head_dim, bool ring, const void *k, const void *v,
                              int64_t n_items_bound, cudaStream_t st);
-cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *q, const void *k, const void *v,
-                             cudaStream_t st);
+cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, cudaStream_t st);
+bool partial_tc_supported(int head_dim, int group, int page_size, int split_keys);
+cudaError_t launch_partial_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, int n_segs,
+                              cudaStream_t st);
 
 constexpr int kArgmaxCluster = 8;
 
