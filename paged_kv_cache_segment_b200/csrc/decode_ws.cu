@@ -56,14 +56,15 @@ struct WsCfg {
     static constexpr int kStageBytes = 2 * kTileBytes;  // K then V
     static constexpr int kStages = D == 256 ? 3 : (D == 128 ? 3 : 6);
     static constexpr int kNQ = 2;
-    static constexpr int kPrefixMax = D == 256 ? 1024 : 256;
+    static constexpr int kPrefixMax = D == 256 ? 512 : 256;
     static constexpr int kMinBlocks = D == 256 ? 1 : 2;
     static constexpr int kQBytes = kWsQ * D * 2;
     static constexpr int kCombBytes = (NC / 2) * kWsQ * D * 4;
     static constexpr int kOffQ = kStages * kStageBytes;
     static constexpr int kOffComb = kOffQ + kNQ * kQBytes;
     static constexpr int kOffPrefix = kOffComb + kCombBytes;
-    static constexpr int kSmem = kOffPrefix + (kPrefixMax + 1) * 4 + 1024;
+    // the stream prefix of items, the prefix of full-split items, the tail order
+    static constexpr int kSmem = kOffPrefix + 3 * (kPrefixMax + 1) * 4 + 1024;
 };
 
 struct WsItem {
@@ -122,24 +123,62 @@ __device__ __forceinline__ int ws_stream_splits(const WsParams &p, int s, uint32
     }
 }
 
+// Work order.  Items are dealt to the CTAs in a snake (round r goes left to
+// right when r is even, right to left when odd) over a balanced order: every
+// stream's full-length splits first, then the streams' last (shorter) splits
+// by decreasing length.  The heavy items spread evenly and the light ones fill
+// the gaps, so the last CTA to finish carries about the average load.
+__device__ __forceinline__ int ws_snake(int k, int bid, int grid) {
+    return k * grid + ((k & 1) ? grid - 1 - bid : bid);
+}
+
+// Keys of stream s's split length, and the number of TK-key tiles its last
+// split takes (0 if the stream has no splits).
 template <bool RING>
-__device__ __forceinline__ WsItem ws_resolve(const WsParams &p, const int *prefix, int L) {
-    // the stream: the last prefix entry <= L
-    int lo = 0, hi = p.n_segs;  // prefix[lo] <= L < prefix[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (prefix[mid] <= L)
-            lo = mid;
-        else
-            hi = mid;
+__device__ __forceinline__ int ws_split_len(const WsParams &p, int s) {
+    if constexpr (RING) {
+        return p.split_keys;
+    } else {
+        int per = p.split_keys;
+        if (per <= 0) {
+            const tf_seg e = p.segs[s];
+            per = (e.n_keys + p.n_splits_max - 1) / p.n_splits_max;
+            per = ((per + (1 << p.log2_page) - 1) >> p.log2_page) << p.log2_page;
+        }
+        return per;
+    }
+}
+
+template <bool RING>
+__device__ __forceinline__ WsItem ws_resolve(const WsParams &p, const int *prefix, const int *prefix_full,
+                                             const int *tail_order, int n_full, int idx) {
+    int lo, g, c;
+    if (idx < n_full) {
+        // a full-length split: the stream is the last prefix_full entry <= idx
+        lo = 0;
+        int hi = p.n_segs;  // prefix_full[lo] <= idx < prefix_full[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (prefix_full[mid] <= idx)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int n_f = (prefix[lo + 1] - prefix[lo]) / p.hkv - 1;  // full splits per kv-head
+        const int r = idx - prefix_full[lo];
+        g = r / n_f;
+        c = r - g * n_f;
+    } else {
+        // a last split, in the tail order
+        const int t = idx - n_full;
+        lo = tail_order[t / p.hkv];
+        g = t % p.hkv;
+        c = (prefix[lo + 1] - prefix[lo]) / p.hkv - 1;
     }
     WsItem it;
     it.s = lo;
-    const int n_units = prefix[lo + 1] - prefix[lo];  // Hkv * n_splits
-    const int n_sp = n_units / p.hkv;
-    const int r = L - prefix[lo];
-    it.g = r / n_sp;
-    it.c = r - it.g * n_sp;
+    it.g = g;
+    it.c = c;
     if constexpr (RING) {
         const tf_ring_seg e = p.rsegs[lo];
         it.q_row = e.q_row;
@@ -196,7 +235,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
     __shared__ uint32_t s_meta[C::kStages];
     __shared__ float comb_m[C::NC / 2][kWsQ], comb_l[C::NC / 2][kWsQ];
     __shared__ uint32_t comb_f[C::NC / 2][kWsQ];
-    __shared__ int s_total;
+    __shared__ int s_total, s_full;
     __shared__ uint32_t s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -204,6 +243,10 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
     const uint32_t sbase = (sraw + 1023u) & ~1023u;
     unsigned char *base_ptr = smem_raw + (sbase - sraw);
     int *prefix = reinterpret_cast<int *>(base_ptr + C::kOffPrefix);
+    int *prefix_full = prefix + (C::kPrefixMax + 1);
+    int *tail_order = prefix_full + (C::kPrefixMax + 1);
+    constexpr int kBuckets = 64;  // tail lengths, in tiles (longer tails share the top bucket)
+    __shared__ int s_bucket[kBuckets];
     float *comb_o = reinterpret_cast<float *>(base_ptr + C::kOffComb);
 
     // ---- prologue: barriers, the item prefix, empty-partial markers
@@ -222,29 +265,80 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
         prefetch_tensormap(&tmV);
     }
     if (warp == 0) {
+        // per stream: its items (splits x Hkv), its full-length ones, and the
+        // tile count of its last split, bucketed for the tail order
         uint32_t bits = 0;
-        int running = 0;
+        int running = 0, running_full = 0;
+        s_bucket[lane] = 0;
+        s_bucket[lane + 32] = 0;
+        __syncwarp();
         for (int b0 = 0; b0 < p.n_segs; b0 += 32) {
             const int s = b0 + lane;
-            const int units = s < p.n_segs ? ws_stream_splits<RING>(p, s, bits) * p.hkv : 0;
-            int incl = units;
+            const int n_sp = s < p.n_segs ? ws_stream_splits<RING>(p, s, bits) : 0;
+            const int units = n_sp * p.hkv, full = n_sp > 0 ? (n_sp - 1) * p.hkv : 0;
+            if (n_sp > 0) {
+                const int n_keys = RING ? p.rsegs[s].n_valid : p.segs[s].n_keys;
+                const int tail = n_keys - (n_sp - 1) * ws_split_len<RING>(p, s);
+                atomicAdd(&s_bucket[min(kBuckets, (tail + C::TK - 1) / C::TK) - 1], 1);
+            }
+            int incl = units, incl_f = full;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
+                const int v = __shfl_up_sync(0xffffffffu, incl, o), vf = __shfl_up_sync(0xffffffffu, incl_f, o);
+                if (lane >= o) {
+                    incl += v;
+                    incl_f += vf;
+                }
             }
-            if (s < p.n_segs) prefix[s] = running + incl - units;
+            if (s < p.n_segs) {
+                prefix[s] = running + incl - units;
+                prefix_full[s] = running_full + incl_f - full;
+            }
             running += __shfl_sync(0xffffffffu, incl, 31);
+            running_full += __shfl_sync(0xffffffffu, incl_f, 31);
         }
+        __syncwarp();
         if (lane == 0) {
             prefix[p.n_segs] = running;
+            prefix_full[p.n_segs] = running_full;
             s_total = running;
+            s_full = running_full;
+            // bucket starts in the tail order, longest tails first
+            int at = 0;
+            for (int k = kBuckets - 1; k >= 0; --k) {
+                const int n = s_bucket[k];
+                s_bucket[k] = at;
+                at += n;
+            }
+        }
+        __syncwarp();
+        // each stream with splits takes the next place of its bucket, streams
+        // in index order within a bucket
+        for (int b0 = 0; b0 < p.n_segs; b0 += 32) {
+            const int s = b0 + lane;
+            int bk = -1;
+            if (s < p.n_segs) {
+                const int units = prefix[s + 1] - prefix[s];
+                if (units > 0) {
+                    const int n_sp = units / p.hkv;
+                    const int n_keys = RING ? p.rsegs[s].n_valid : p.segs[s].n_keys;
+                    const int tail = n_keys - (n_sp - 1) * ws_split_len<RING>(p, s);
+                    bk = min(kBuckets, (tail + C::TK - 1) / C::TK) - 1;
+                }
+            }
+            const uint32_t same = __match_any_sync(0xffffffffu, bk);
+            const int rank = __popc(same & ((1u << lane) - 1u));
+            if (bk >= 0) tail_order[s_bucket[bk] + rank] = s;
+            __syncwarp();
+            if (bk >= 0 && rank == 0) s_bucket[bk] += __popc(same);
+            __syncwarp();
         }
         bits |= __reduce_or_sync(0xffffffffu, bits);
         if (lane == 0 && bits && blockIdx.x == 0) atomicOr(p.status, bits);
     }
     __syncthreads();
-    const int total = s_total;
+    const int total = s_total, n_full = s_full;
+    const int bid = (int)blockIdx.x, grid = (int)gridDim.x;
 
     if (warp == C::NC) {
         // ---- producer warp
@@ -283,20 +377,20 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             };
             uint32_t tc = 0, qc = 0;
             bool ok = true;
-            int L = blockIdx.x;
+            int k = 0, L = ws_snake(0, bid, grid);
             WsItem it{};
             int win = 0, w0 = 0;
             if (L < total) {
-                it = ws_resolve<RING>(p, prefix, L);
+                it = ws_resolve<RING>(p, prefix, prefix_full, tail_order, n_full, L);
                 w0 = it.key_lo >> p.log2_page;
                 win = load_window(it, w0);
             }
             while (L < total && ok) {
-                const int L_next = L + (int)gridDim.x;
+                const int L_next = ws_snake(k + 1, bid, grid);
                 WsItem nx{};
                 int win_next = 0, w0_next = 0;
                 if (L_next < total) {  // requested now, used when the next item starts
-                    nx = ws_resolve<RING>(p, prefix, L_next);
+                    nx = ws_resolve<RING>(p, prefix, prefix_full, tail_order, n_full, L_next);
                     w0_next = nx.key_lo >> p.log2_page;
                     win_next = load_window(nx, w0_next);
                 }
@@ -380,6 +474,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                     j0 += rows;
                 }
                 L = L_next;
+                ++k;
                 it = nx;
                 win = win_next;
                 w0 = w0_next;
@@ -397,8 +492,8 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
     const int gq = lane >> 2, t4 = lane & 3;
     const float scale_log2 = p.scale_log2;
     uint32_t tc = 0, qc = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x) {
-        const WsItem it = ws_resolve<RING>(p, prefix, L);
+    for (int k = 0, L = ws_snake(0, bid, grid); L < total; L = ws_snake(++k, bid, grid)) {
+        const WsItem it = ws_resolve<RING>(p, prefix, prefix_full, tail_order, n_full, L);
         const int q_item = it.n_rows * p.group;
         // queries of this item -> B fragments (Q^T), kept in registers
         const uint32_t qs = qc % C::kNQ;
