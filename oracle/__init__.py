@@ -54,6 +54,7 @@ class Oracle:
         L.orc_gather_paged.argtypes = [P, P, i32, i32, i32, i32, P, i32, i32, i32, P, P]
         L.orc_gather_paged.restype = ctypes.c_int
         L.orc_paged_attn.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, i32, f64, i32, P, P, P]
+        L.orc_put_rows.argtypes = [P, P, i32, i32, i32, P, P, i32, i32, P, i32, P, i32]
         L.orc_paged_attn.restype = ctypes.c_int
         L.orc_partial.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, P, P, P, P]
         L.orc_partial.restype = None
@@ -92,6 +93,24 @@ class Oracle:
                                        pt_base, n_stream_pages, n_keys, self._p(kd), self._p(vd))
         self._check(rc, "gather")
         return kd, vd
+
+    # ------------------------------------------------------- rows into pages
+    def put_rows(self, k_rows, v_rows, k_pool, v_pool, page_table, segs):
+        """Copies of the pools with each stream's new rows written into its pages
+        (orc_put_rows); k_rows, v_rows bf16 bits [rows][Hkv][D]."""
+        k_rows = np.ascontiguousarray(k_rows, np.uint16)
+        v_rows = np.ascontiguousarray(v_rows, np.uint16)
+        kp = np.array(k_pool, np.uint16, copy=True, order="C")
+        vp = np.array(v_pool, np.uint16, copy=True, order="C")
+        pt = np.ascontiguousarray(page_table, np.int32)
+        segs = np.ascontiguousarray(segs, np.int32).reshape(-1, 5)
+        rows, hkv, d = k_rows.shape
+        n_pages, hkv2, psz, d2 = kp.shape
+        assert (hkv, d) == (hkv2, d2) and v_rows.shape == k_rows.shape
+        rc = self.lib.orc_put_rows(self._p(k_rows), self._p(v_rows), rows, hkv, d, self._p(kp), self._p(vp), n_pages,
+                                   psz, self._p(pt), len(pt), self._p(segs), len(segs))
+        self._check(rc, "put_rows")
+        return kp, vp
 
     # ------------------------------------------------------- paged attention
     def paged_attn(self, q, k_pool, v_pool, page_table, segs, scale, full=False, sel=None):

@@ -35,6 +35,9 @@
  *         segment from a table; slots are stepped with a wrap.
  *  [ARG]  #1503, commit list: lfm2_argmax picks each row's first largest
  *         logit, ties to the lower id, and flags a row with a nonfinite logit.
+ *  [WR]   #1653, PR body: the rows kernel writes a stream's new K/V rows and
+ *         tf_wrows_put copies them into the stream's pages; forward refuses
+ *         rows past a slot's pages (PastPages).
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - pool layout [page][kv_head][slot][D], K and V in separate arrays;
@@ -165,7 +168,9 @@ int orc_paged_attn(const uint16_t *q, int32_t n_rows_total, int32_t n_q_heads, c
     for (int32_t s = 0; s < n_segs; ++s) {
         const int32_t q_row = segs[5 * s + 0], n_rows = segs[5 * s + 1], n_keys = segs[5 * s + 2];
         const int32_t pt_base = segs[5 * s + 3], n_pg = segs[5 * s + 4];
-        if (q_row < 0 || n_rows < 0 || q_row + n_rows > n_rows_total || n_keys < n_rows || pt_base < 0 ||
+        /* the causal count needs a key per row; a FULL block row needs one key */
+        const int32_t keys_needed = full ? (n_rows > 0 ? 1 : 0) : n_rows;
+        if (q_row < 0 || n_rows < 0 || q_row + n_rows > n_rows_total || n_keys < keys_needed || pt_base < 0 ||
             n_pg < 0 || pt_base + n_pg > pt_len)
             return ORC_ERR_ARG;
         if (n_rows == 0) continue;
@@ -204,6 +209,54 @@ int orc_paged_attn(const uint16_t *q, int32_t n_rows_total, int32_t n_q_heads, c
         }
         free(kd);
         free(vd);
+    }
+    return ORC_OK;
+}
+
+/*
+ * A stream's new rows into its pages ([WR]).  Row i of segment s is the
+ * stream's key j = n_keys - n_rows + i (its new rows are its last keys); for
+ * every kv-head g its K row and V row are copied to slot j % page_size of page
+ * page_table[pt_base + j / page_size]:
+ *     k_pool[page][g][slot][:] = k_rows[q_row + i][g][:]   (same for v).
+ * Every entry is checked before anything is copied: a bad entry gives
+ * ORC_ERR_ARG, a key past the stream's pages ORC_ERR_PAST_PAGES, a page id
+ * out of range ORC_ERR_BAD_PAGE, and the pools are then left as they were.
+ */
+int orc_put_rows(const uint16_t *k_rows, const uint16_t *v_rows, int32_t n_rows_total, int32_t n_kv_heads,
+                 int32_t head_dim, uint16_t *k_pool, uint16_t *v_pool, int32_t n_pages, int32_t page_size,
+                 const int32_t *page_table, int32_t pt_len, const int32_t *segs, int32_t n_segs)
+{
+    if (n_kv_heads <= 0 || head_dim <= 0 || page_size <= 0) return ORC_ERR_ARG;
+    for (int32_t s = 0; s < n_segs; ++s) {
+        const int32_t q_row = segs[5 * s + 0], n_rows = segs[5 * s + 1], n_keys = segs[5 * s + 2];
+        const int32_t pt_base = segs[5 * s + 3], n_pg = segs[5 * s + 4];
+        if (q_row < 0 || n_rows < 0 || q_row + n_rows > n_rows_total || n_keys < n_rows || pt_base < 0 ||
+            n_pg < 0 || pt_base + n_pg > pt_len)
+            return ORC_ERR_ARG;
+        if ((int64_t)n_keys > (int64_t)n_pg * page_size) return ORC_ERR_PAST_PAGES;
+        for (int32_t i = 0; i < n_rows; ++i) {
+            const int32_t j = n_keys - n_rows + i;
+            const int32_t pid = page_table[pt_base + j / page_size];
+            if (pid < 0 || pid >= n_pages) return ORC_ERR_BAD_PAGE;
+        }
+    }
+    for (int32_t s = 0; s < n_segs; ++s) {
+        const int32_t q_row = segs[5 * s + 0], n_rows = segs[5 * s + 1], n_keys = segs[5 * s + 2];
+        const int32_t pt_base = segs[5 * s + 3];
+        for (int32_t i = 0; i < n_rows; ++i) {
+            const int32_t j = n_keys - n_rows + i;
+            const int64_t page = page_table[pt_base + j / page_size];
+            const int64_t slot = j % page_size;
+            for (int32_t g = 0; g < n_kv_heads; ++g) {
+                const int64_t src = ((int64_t)(q_row + i) * n_kv_heads + g) * head_dim;
+                const int64_t dst = ((page * n_kv_heads + g) * page_size + slot) * head_dim;
+                for (int32_t d = 0; d < head_dim; ++d) {
+                    k_pool[dst + d] = k_rows[src + d];
+                    v_pool[dst + d] = v_rows[src + d];
+                }
+            }
+        }
     }
     return ORC_OK;
 }

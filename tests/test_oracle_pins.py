@@ -36,9 +36,10 @@ def bf16_round(x):
     return wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(np.asarray(x, np.float32))).astype(np.float64)
 
 
-def scatter_into_pages(k_dense_bits, v_dense_bits, page_size, n_pool, rng, poison=True):
+def scatter_into_pages(k_dense_bits, v_dense_bits, page_size, n_pool, rng, poison=True, reserve=None):
     """Write each stream's keys into pages drawn from a shuffled pool:
-    key j goes to page table entry j // P, slot j % P.  Returns pool, table, segs."""
+    key j goes to page table entry j // P, slot j % P.  `reserve` (per stream)
+    takes at least that many pages for a stream.  Returns pool, table, segs."""
     hkv, d = k_dense_bits[0].shape[1:]
     shape = (n_pool, hkv, page_size, d)
     fill = wl.BF16_NAN if poison else np.uint16(0)
@@ -48,9 +49,9 @@ def scatter_into_pages(k_dense_bits, v_dense_bits, page_size, n_pool, rng, poiso
     table = []
     nxt = 0
     bases = []
-    for kd, vd in zip(k_dense_bits, v_dense_bits):
+    for si, (kd, vd) in enumerate(zip(k_dense_bits, v_dense_bits)):
         n = kd.shape[0]
-        npg = -(-n // page_size)
+        npg = max(-(-n // page_size), reserve[si] if reserve is not None else 0)
         bases.append((len(table), npg))
         pages = perm[nxt:nxt + npg]
         nxt += npg
@@ -120,6 +121,86 @@ def test_full_flag_matches_sdpa_without_mask(orc):
                              wl.bf16_bits_to_f32(kd).astype(np.float64), wl.bf16_bits_to_f32(vd).astype(np.float64),
                              0.3, r, n, full=True)
         np.testing.assert_allclose(out[r0:r0 + r], ref, rtol=0, atol=TOL)
+
+
+def test_full_block_may_be_longer_than_its_keys(orc):
+    """[FULL]: a drafter block of up to nine rows over the keys [0, len + 1)
+    may hold more rows than keys; every row sees them all."""
+    rows, keys = [9, 3], [3, 1]
+    q, ks, vs, kp, vp, table, segs = make_streams(6, rows, keys, 4, 2, 32, 8)
+    out, flags = orc.paged_attn(q, kp, vp, table, segs, 0.25, full=True)
+    assert not flags.any()
+    for (r0, r, n, _, _), kd, vd in zip(segs, ks, vs):
+        ref = sdpa_reference(wl.bf16_bits_to_f32(q[r0:r0 + r]).astype(np.float64),
+                             wl.bf16_bits_to_f32(kd).astype(np.float64), wl.bf16_bits_to_f32(vd).astype(np.float64),
+                             0.25, r, n, full=True)
+        np.testing.assert_allclose(out[r0:r0 + r], ref, rtol=0, atol=TOL)
+    with pytest.raises(ValueError):  # the causal count needs a key per row
+        orc.paged_attn(q, kp, vp, table, segs, 0.25)
+
+
+def append_case(seed, rows, keys, hkv, d, p, extra=3):
+    """Streams of N keys whose last R keys arrive as new rows: the pools before
+    (first N - R keys written, the rest NaN), the pools a writer gives with all N
+    keys in place, the rows [sum R][Hkv][D] and the segment table."""
+    rng = np.random.default_rng(seed)
+    ks = [wl.normal_bf16(rng, (n, hkv, d)) for n in keys]
+    vs = [wl.normal_bf16(rng, (n, hkv, d)) for n in keys]
+    n_pool = sum(-(-n // p) for n in keys) + extra
+    reserve = [-(-n // p) for n in keys]
+    kp_all, vp_all, table, bases = scatter_into_pages(ks, vs, p, n_pool, np.random.default_rng(seed + 1),
+                                                      reserve=reserve)
+    kp_old, vp_old, table2, _ = scatter_into_pages([k[:n - r] for k, n, r in zip(ks, keys, rows)],
+                                                   [v[:n - r] for v, n, r in zip(vs, keys, rows)], p, n_pool,
+                                                   np.random.default_rng(seed + 1), reserve=reserve)
+    assert np.array_equal(table, table2)
+    k_rows = np.concatenate([k[n - r:] for k, n, r in zip(ks, keys, rows)])
+    v_rows = np.concatenate([v[n - r:] for v, n, r in zip(vs, keys, rows)])
+    segs, r0 = [], 0
+    for (b, npg), r, n in zip(bases, rows, keys):
+        segs.append((r0, r, n, b, npg))
+        r0 += r
+    return kp_old, vp_old, kp_all, vp_all, k_rows, v_rows, table, np.array(segs, np.int32)
+
+
+@pytest.mark.parametrize("rows,keys,hkv,d,p", [([3, 1, 5], [37, 8, 40], 2, 16, 8), ([16], [16], 1, 8, 4),
+                                               ([2, 7], [33, 64], 3, 32, 32)])
+def test_put_rows_matches_the_writer(orc, rows, keys, hkv, d, p):
+    """[WR]: putting the new rows gives byte for byte the pools a writer that
+    placed every key from the start gives, and nothing else changes."""
+    kp_old, vp_old, kp_all, vp_all, kr, vr, table, segs = append_case(21 + d, rows, keys, hkv, d, p)
+    kp, vp = orc.put_rows(kr, vr, kp_old, vp_old, table, segs)
+    assert np.array_equal(kp, kp_all) and np.array_equal(vp, vp_all)
+    changed = int((kp != kp_old).sum() + (vp != vp_old).sum())
+    assert changed == 2 * sum(rows) * hkv * d  # every named slot, nothing more
+
+
+def test_gather_after_put_returns_the_rows(orc):
+    rows, keys, hkv, d, p = [4, 1], [21, 9], 2, 16, 8
+    kp_old, vp_old, _, _, kr, vr, table, segs = append_case(3, rows, keys, hkv, d, p)
+    kp, vp = orc.put_rows(kr, vr, kp_old, vp_old, table, segs)
+    for (r0, r, n, b, npg) in segs:
+        kd, vd = orc.gather_paged(kp, vp, table, b, npg, n)
+        k0, v0 = orc.gather_paged(kp_old, vp_old, table, b, npg, n)
+        np.testing.assert_array_equal(kd[n - r:], wl.bf16_bits_to_f32(kr[r0:r0 + r]).astype(np.float64))
+        np.testing.assert_array_equal(vd[n - r:], wl.bf16_bits_to_f32(vr[r0:r0 + r]).astype(np.float64))
+        np.testing.assert_array_equal(kd[:n - r], k0[:n - r])  # earlier keys untouched
+
+
+def test_put_rows_refusals(orc):
+    kp_old, vp_old, _, _, kr, vr, table, segs = append_case(4, [2], [10], 1, 8, 4)
+    past = segs.copy()
+    past[0, 2] = past[0, 4] * 4 + 1  # a key past the stream's pages
+    with pytest.raises(ValueError, match="past"):
+        orc.put_rows(kr, vr, kp_old, vp_old, table, past)
+    bad_table = table.copy()
+    bad_table[segs[0, 3] + 2] = kp_old.shape[0]  # the page of keys 8..9 outside the pool
+    with pytest.raises(ValueError, match="page id"):
+        orc.put_rows(kr, vr, kp_old, vp_old, bad_table, segs)
+    short = segs.copy()
+    short[0, 2] = 1  # fewer keys than new rows
+    with pytest.raises(ValueError):
+        orc.put_rows(kr, vr, kp_old, vp_old, table, short)
 
 
 def test_gather_is_the_writer_inverse(orc):
@@ -439,6 +520,8 @@ CONTROLS = {
     "merge_weight_dropped": ("if (l[c] > 0.0) denom += exp(m[c] - mx) * l[c];", "if (l[c] > 0.0) denom += l[c];"),
     "ring_no_lag": ("int32_t slot = ((e.head - n + j) % e.size + e.size) % e.size;",
                     "int32_t slot = ((e.head + j) % e.size + e.size) % e.size;"),
+    "put_rows_reversed": ("const int32_t j = n_keys - n_rows + i;\n            const int64_t page",
+                          "const int32_t j = n_keys - 1 - i;\n            const int64_t page"),
 }
 
 
@@ -470,6 +553,7 @@ PIN_FOR = {
     "gqa_modulo": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
     "merge_weight_dropped": lambda o: test_merged_partials_equal_unsplit(o, 0),
     "ring_no_lag": lambda o: test_ring_matches_a_writer(o, 10, 13, 6),
+    "put_rows_reversed": lambda o: test_put_rows_matches_the_writer(o, [3, 1, 5], [37, 8, 40], 2, 16, 8),
 }
 
 
