@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--only", default="", help="comma list: decode,verify,ring,prompt,argmax,e2e,cpu")
+    ap.add_argument("--only", default="", help="comma list: decode,verify,ring,prompt,argmax,block,append,e2e,cpu")
     ap.add_argument("--secondary-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -365,6 +365,10 @@ def run_native(args):
             sec["ring"] = bench_ring(wl, tf, dev, ks, peaks, traffic)
         if want(args, "prompt"):
             sec["prompt"] = bench_prompt(wl, tf, dev, max(3, ks // 4), peaks)
+        if want(args, "block"):
+            sec["block"] = bench_block(wl, tf, dev, ks, peaks)
+        if want(args, "append"):
+            sec["append"] = bench_append(wl, tf, dev, ks, peaks)
         result["secondary"] = sec
         result["gpu_launches_secondary"] = sum(v.get("launches", 0) for v in sec.values())
     if rank == 0 and world == 1 and want(args, "cpu"):
@@ -515,6 +519,78 @@ def bench_prompt(wl, tf, dev, steps, peaks):
             "algorithmic_flops": flops,
             "roofline": roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s"), "launches": len(segs) * steps,
             "l2": "2 rotating copies"}
+
+
+def bench_block(wl, tf, dev, steps, peaks):
+    """A drafter-block round: 16 streams, each a block of 9 rows seeing all of
+    its stream's keys (the FULL rule), contexts U{1,024..8,192}, 32/8 heads,
+    D 128, pages of 32, 512-key partials + merge; 3 rotating copies."""
+    import torch
+
+    b0 = wl.multi_stream_decode(2)
+    keys = [int(x) for x in b0.segs[:, 2]]
+    b = wl.make_paged_batch(12, [9] * len(keys), keys, 32, 8, 128, 32, unused="nan", split_keys=512)
+    run = DecodeRun(b, dev)
+
+    def step(k):
+        x = run.sets[k % len(run.sets)]
+        tf.tf_paged_attn_block(x["q"], x["kp"], x["vp"], x["pt"], x["segs"], scale=b.scale,
+                               split_keys=b.split_keys, n_splits_max=b.n_splits_max, part_o=run.po, part_m=run.pm,
+                               part_l=run.pl, part_flag=run.pf, status=run.st, segs_host=b.segs)
+        run.merge(k)
+
+    for k in range(3):
+        step(k)
+    _, total = timed_steps([step], steps)
+    ms = total / steps
+    kv = b.kv_bytes()
+    assert int(run.st.item()) == 0
+    return {"workload": "drafter blocks: 16 streams x 9 rows, every row over all its stream's keys, contexts "
+                        "U{1024..8192}, 32/8 heads, D128, P32, 512-key partials + merge",
+            "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2), "ms_per_step": round(ms, 5),
+            "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"),
+                             kernel="prompt_tc_kernel<128, hilo, partial> + merge (the whole step)"),
+            "launches": 2 * steps, "l2": "3 rotating copies"}
+
+
+def bench_append(wl, tf, dev, steps, peaks):
+    """The 15,000-token prompt's keys and values appended in one call (4
+    kv-heads, D 256, pages of 32) into a shuffled pool; 3 rotating pool
+    copies.  Bytes: every row read once from the row arrays and written once
+    into the pools."""
+    import torch
+
+    b, _ = wl.long_prompt(4)
+    n, hkv, d = b.n_rows_total, b.n_kv_heads, b.head_dim
+    rng = np.random.default_rng(13)
+    kr = to_dev(wl.normal_bf16(rng, (n, hkv, d)), dev)
+    vr = to_dev(wl.normal_bf16(rng, (n, hkv, d)), dev)
+    pools = [(to_dev(b.k_pool, dev), to_dev(b.v_pool, dev)) for _ in range(3)]
+    pt = to_dev(b.page_table, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    seg = b.segs[0]
+    # one call over all rows: the kernel's own rate (chunk-sized calls of a
+    # few microseconds each would time the host's launch path instead)
+    sh = np.array([[0, n, n, seg[3], seg[4]]], np.int32)
+    calls = [(sh, to_dev(sh, dev))]
+
+    def step(k):
+        kp, vp = pools[k % 3]
+        for sh, sd in calls:
+            tf.tf_kv_append(kr, vr, kp, vp, pt, sd, status=st, segs_host=sh)
+
+    for k in range(3):
+        step(k)
+    _, total = timed_steps([step], steps)
+    ms = total / steps
+    moved = 2 * 2 * n * hkv * d * 2  # K and V, read from the rows and written into the pages
+    assert int(st.item()) == 0
+    gbs = moved / (ms * 1e-3) / 1e9
+    return {"workload": "append the 15,000-token prompt's K/V rows into 469 shuffled pages of 32 in one call "
+                        "(4 kv-heads, D256)", "gbs": round(gbs, 2), "ms_per_step": round(ms, 5),
+            "bytes_per_step": moved, "roofline": dict(roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
+                                                      kernel="kv_append_kernel<256>"),
+            "launches": len(calls) * steps, "l2": "3 rotating pool copies (rows arrays resident)"}
 
 
 def cpu_baseline(b, seconds):

@@ -144,6 +144,54 @@ TF_API tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32
                                uint8_t *part_flag, uint32_t *status, tf_stream_t stream);
 
 /*
+ * tf_paged_attn_decode with the FULL rule of #1394 ("lfm2: a cheaper DSpark
+ * hold", commit list: the block attention and merge kernels with a FULL
+ * template flag): every row of a stream sees all of its stream's keys
+ * [0, n_keys) instead of the causal count, as a drafter block (the pending
+ * token and its mask tokens) attends over the context keys [0, len + 1).
+ * Arguments, layouts, outputs and errors are those of tf_paged_attn_decode,
+ * except that a stream may have more rows than keys (at least one key when it
+ * has rows).  The partials merge with tf_attn_merge.
+ */
+TF_API tf_status tf_paged_attn_block(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                              const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                              int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                              const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                              const int32_t *page_table_host, float scale, int32_t split_keys,
+                              int32_t n_splits_max, float *part_o, float *part_m, float *part_l,
+                              uint8_t *part_flag, uint32_t *status, tf_stream_t stream);
+
+/*
+ * Append each stream's new rows' keys and values into its pages: the
+ * counterpart of tf_wrows_put in #1653 ("spark25 CUDA: the full layers'
+ * caches in pages of the core pool", PR body: the rows kernel writes kr/vr
+ * and tf_wrows_put copies them into the pages; forward refuses rows past a
+ * slot's pages, PastPages).
+ *
+ * Row i (0 <= i < n_rows) of stream s is key j = n_keys - n_rows + i of that
+ * stream (a stream's new rows are its last keys, the convention of every
+ * attention call here).  For every kv-head g:
+ *   k_pool[page][g][j % page_size][:] = k_rows[q_row + i][g][:], same for v,
+ *   page = page_table[pt_base + j / page_size].
+ * Nothing else in the pools changes.
+ *
+ *  k_rows, v_rows  bf16 [n_rows_total][n_kv_heads][head_dim], 16-byte aligned
+ *  k_pool, v_pool  bf16 [n_pages][n_kv_heads][page_size][head_dim] (written)
+ *  page_table, segs, segs_host, page_table_host, status: as for
+ *             tf_paged_attn_decode; a row whose key lies past the stream's
+ *             pages (TF_ERR_PAST_PAGES from the host check, TF_DEV_PAST_PAGES
+ *             on the device) or whose page id is out of range
+ *             (TF_ERR_BAD_PAGE / TF_DEV_BAD_PAGE) is not written.
+ * Streams must not share pages for the rows they write (two writes to one
+ * slot race).  Supported head dims and page sizes: as tf_paged_attn_decode.
+ */
+TF_API tf_status tf_kv_append(const void *k_rows, const void *v_rows, int32_t n_rows_total, void *k_pool,
+                              void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                              int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                              const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                              const int32_t *page_table_host, uint32_t *status, tf_stream_t stream);
+
+/*
  * Fold partials into the final output (the merge bodies of #1503, commit
  * list; the nonfinite-head handling of #1653, review thread).  Per (row, head):
  * M = max m_c over partials with l_c > 0, L = sum e^(m_c - M) l_c,

@@ -14,6 +14,8 @@ from .binding import (  # noqa: F401
     tf_abi_version,
     tf_argmax_rows,
     tf_attn_merge,
+    tf_kv_append,
+    tf_paged_attn_block,
     tf_paged_attn_decode,
     tf_paged_attn_prompt,
     tf_ring_attn,

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "TF_OK", 1: "TF_ERR_ARG", 2: "TF_ERR_PAST_PAGES", 3: "TF_ERR_
 TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS = 1, 2, 4, 8
 TF_OUT_F32, TF_OUT_BF16 = 0, 1
 
-EXPORTS = ("tf_paged_attn_decode", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
+EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
            "tf_ring_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_status_str", "tf_abi_version")
 # bytes of the scratch array tf_ring_attn_noalloc keeps in the library's device image
 TF_RING_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     lib.tf_paged_attn_decode.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, i32, P, P, f32, i32, i32,
                                          P, P, P, P, P, P]
+    lib.tf_paged_attn_block.argtypes = lib.tf_paged_attn_decode.argtypes
+    lib.tf_kv_append.argtypes = [P, P, i32, P, P, i32, i32, i32, i32, P, i32, P, i32, P, P, P, P]
     lib.tf_attn_merge.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P]
     lib.tf_paged_attn_prompt.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, f32, P, i32, P, P, P]
     lib.tf_ring_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, f32, i32, i32, P, sz, P, P, P, P]
@@ -65,7 +67,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_status_str.argtypes = [ctypes.c_int]
     lib.tf_status_str.restype = ctypes.c_char_p
     lib.tf_abi_version.restype = ctypes.c_int32
-    for name in ("tf_paged_attn_decode", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
+    for name in ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
                  "tf_ring_attn_noalloc", "tf_argmax_rows"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -141,6 +143,44 @@ def tf_paged_attn_decode(q, k_pool, v_pool, page_table, segs, *, scale, split_ke
         _dev(part_l, "part_l", (torch.float32,)), _dev(part_flag, "part_flag", (torch.uint8,)),
         _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
     _check("tf_paged_attn_decode", rc)
+
+
+def tf_paged_attn_block(q, k_pool, v_pool, page_table, segs, *, scale, split_keys, n_splits_max, part_o, part_m,
+                        part_l, part_flag, status, segs_host=None, page_table_host=None, stream=None):
+    """Split-KV partials where every row sees all of its stream's keys (tf_paged_attn_block)."""
+    lib = load()
+    rows, hq, d = q.shape
+    n_pages, hkv, psz, d2 = k_pool.shape
+    if d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("q / pool head dims disagree")
+    sh = as_segs_np(segs_host) if segs_host is not None else None
+    pth = np.ascontiguousarray(np.asarray(page_table_host, np.int32)) if page_table_host is not None else None
+    rc = lib.tf_paged_attn_block(
+        _dev(q, "q", BF16), rows, hq, _dev(k_pool, "k_pool", BF16), _dev(v_pool, "v_pool", BF16), n_pages, psz, hkv, d,
+        _dev(page_table, "page_table", (torch.int32,)), page_table.numel(), _dev(segs, "segs", (torch.int32,)),
+        segs.numel() // 5, _host_ptr(sh), _host_ptr(pth), float(scale), int(split_keys), int(n_splits_max),
+        _dev(part_o, "part_o", (torch.float32,)), _dev(part_m, "part_m", (torch.float32,)),
+        _dev(part_l, "part_l", (torch.float32,)), _dev(part_flag, "part_flag", (torch.uint8,)),
+        _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
+    _check("tf_paged_attn_block", rc)
+
+
+def tf_kv_append(k_rows, v_rows, k_pool, v_pool, page_table, segs, *, status, segs_host=None, page_table_host=None,
+                 stream=None):
+    """Each stream's new rows [rows][Hkv][D] into their pages (tf_kv_append)."""
+    lib = load()
+    rows, hkv, d = k_rows.shape
+    n_pages, hkv2, psz, d2 = k_pool.shape
+    if (hkv2, d2) != (hkv, d) or tuple(v_pool.shape) != tuple(k_pool.shape) or tuple(v_rows.shape) != tuple(k_rows.shape):
+        raise ValueError("rows / pool shapes disagree")
+    sh = as_segs_np(segs_host) if segs_host is not None else None
+    pth = np.ascontiguousarray(np.asarray(page_table_host, np.int32)) if page_table_host is not None else None
+    rc = lib.tf_kv_append(
+        _dev(k_rows, "k_rows", BF16), _dev(v_rows, "v_rows", BF16), rows, _dev(k_pool, "k_pool", BF16),
+        _dev(v_pool, "v_pool", BF16), n_pages, psz, hkv, d, _dev(page_table, "page_table", (torch.int32,)),
+        page_table.numel(), _dev(segs, "segs", (torch.int32,)), segs.numel() // 5, _host_ptr(sh), _host_ptr(pth),
+        _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
+    _check("tf_kv_append", rc)
 
 
 def tf_attn_merge(part_o, part_m, part_l, part_flag, out, flags, *, stream=None):

@@ -32,11 +32,13 @@ int split_len(int n_keys, int split_keys, int n_splits_max, int page_size) {
 
 // Checks of a host copy of a segment table; see tf_paged_attn_decode.
 tf_status check_segs_host(const tf_seg *sh, int n_segs, int n_rows_total, int page_table_len, int page_size,
-                          int n_pages, const int32_t *pt_host, int split_keys, int n_splits_max, int *max_rows) {
+                          int n_pages, const int32_t *pt_host, int split_keys, int n_splits_max, int *max_rows,
+                          bool full = false) {
     int mr = 0;
     for (int s = 0; s < n_segs; ++s) {
         const tf_seg e = sh[s];
-        if (e.q_row < 0 || e.n_rows < 0 || (int64_t)e.q_row + e.n_rows > n_rows_total || e.n_keys < e.n_rows ||
+        if (e.q_row < 0 || e.n_rows < 0 || (int64_t)e.q_row + e.n_rows > n_rows_total ||
+            e.n_keys < (full ? (e.n_rows > 0 ? 1 : 0) : e.n_rows) ||
             e.pt_base < 0 || e.n_pages < 0 || (int64_t)e.pt_base + e.n_pages > page_table_len)
             return TF_ERR_ARG;
         if ((int64_t)e.n_keys > (int64_t)e.n_pages * page_size) return TF_ERR_PAST_PAGES;
@@ -79,9 +81,9 @@ tf_status ring_merge(const float *po, const float *pm, const float *pl, const ui
 
 }  // namespace
 
-extern "C" {
-
-tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+// Split-KV partials of every row of every stream (the causal count, or with
+// `full` every row over all of its stream's keys).
+static tf_status paged_partials(bool full, const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
                                const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
                                int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
                                const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
@@ -105,7 +107,7 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
     int max_rows = n_rows_total;
     if (segs_host) {
         const tf_status st = check_segs_host(segs_host, n_segs, n_rows_total, page_table_len, page_size, n_pages,
-                                             page_table_host, split_keys, n_splits_max, &max_rows);
+                                             page_table_host, split_keys, n_splits_max, &max_rows, full);
         if (st != TF_OK) return st;
         if (max_rows == 0) return TF_OK;
     }
@@ -140,6 +142,7 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
         w.scale_log2 = scale * 1.4426950408889634f;
         w.split_keys = split_keys;
         w.n_splits_max = n_splits_max;
+        w.full = full ? 1 : 0;
         w.part_o = part_o;
         w.part_m = part_m;
         w.part_l = part_l;
@@ -170,6 +173,7 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
             t.split_keys = split_keys;
             t.n_splits_max = n_splits_max;
             t.n_qt = (int)n_qt;
+            t.full = full ? 1 : 0;
             t.part_o = part_o;
             t.part_m = part_m;
             t.part_l = part_l;
@@ -197,6 +201,7 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
     p.split_keys = split_keys;
     p.n_splits_max = n_splits_max;
     p.n_qgroups = (int)n_qgroups;
+    p.full = full ? 1 : 0;
     p.part_o = part_o;
     p.part_m = part_m;
     p.part_l = part_l;
@@ -204,6 +209,69 @@ tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_
     p.status = status;
     const dim3 grid((unsigned)n_splits_max, (unsigned)(n_qgroups * n_kv_heads), (unsigned)n_segs);
     return cuda_status(launch_attn_partial(p, head_dim, false, false, grid, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" {
+
+tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                               const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                               int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                               const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                               const int32_t *page_table_host, float scale, int32_t split_keys,
+                               int32_t n_splits_max, float *part_o, float *part_m, float *part_l,
+                               uint8_t *part_flag, uint32_t *status, tf_stream_t stream) {
+    return paged_partials(false, q, n_rows_total, n_q_heads, k_pool, v_pool, n_pages, page_size, n_kv_heads,
+                          head_dim, page_table, page_table_len, segs, n_segs, segs_host, page_table_host, scale,
+                          split_keys, n_splits_max, part_o, part_m, part_l, part_flag, status, stream);
+}
+
+tf_status tf_paged_attn_block(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                              const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                              int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                              const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                              const int32_t *page_table_host, float scale, int32_t split_keys,
+                              int32_t n_splits_max, float *part_o, float *part_m, float *part_l,
+                              uint8_t *part_flag, uint32_t *status, tf_stream_t stream) {
+    return paged_partials(true, q, n_rows_total, n_q_heads, k_pool, v_pool, n_pages, page_size, n_kv_heads,
+                          head_dim, page_table, page_table_len, segs, n_segs, segs_host, page_table_host, scale,
+                          split_keys, n_splits_max, part_o, part_m, part_l, part_flag, status, stream);
+}
+
+tf_status tf_kv_append(const void *k_rows, const void *v_rows, int32_t n_rows_total, void *k_pool, void *v_pool,
+                       int32_t n_pages, int32_t page_size, int32_t n_kv_heads, int32_t head_dim,
+                       const int32_t *page_table, int32_t page_table_len, const tf_seg *segs, int32_t n_segs,
+                       const tf_seg *segs_host, const int32_t *page_table_host, uint32_t *status,
+                       tf_stream_t stream) {
+    if (n_rows_total < 0 || n_kv_heads <= 0 || n_pages < 0 || page_table_len < 0 || n_segs < 0) return TF_ERR_ARG;
+    if (!head_dim_ok(head_dim)) return TF_ERR_UNSUPPORTED;
+    const int lp = log2_exact(page_size);
+    if (lp < 3 || lp > 10) return TF_ERR_UNSUPPORTED;
+    if (n_segs > 65535) return TF_ERR_UNSUPPORTED;
+    if (n_segs == 0 || n_rows_total == 0) return TF_OK;
+    if (!k_rows || !v_rows || !k_pool || !v_pool || !page_table || !segs || !status) return TF_ERR_ARG;
+    if (!aligned16(k_rows) || !aligned16(v_rows) || !aligned16(k_pool) || !aligned16(v_pool)) return TF_ERR_ALIGN;
+    int max_rows = n_rows_total;
+    if (segs_host) {
+        const tf_status st = check_segs_host(segs_host, n_segs, n_rows_total, page_table_len, page_size, n_pages,
+                                             page_table_host, 0, 0, &max_rows);
+        if (st != TF_OK) return st;
+        if (max_rows == 0) return TF_OK;
+    }
+    if ((int64_t)max_rows * n_kv_heads > ((int64_t)1 << 34)) return TF_ERR_UNSUPPORTED;
+    AppendParams p{};
+    p.k_rows = static_cast<const uint16_t *>(k_rows);
+    p.v_rows = static_cast<const uint16_t *>(v_rows);
+    p.k_pool = static_cast<uint16_t *>(k_pool);
+    p.v_pool = static_cast<uint16_t *>(v_pool);
+    p.n_rows_total = n_rows_total;
+    p.hkv = n_kv_heads;
+    p.n_pages = n_pages;
+    p.log2_page = lp;
+    p.pt_len = page_table_len;
+    p.page_table = page_table;
+    p.segs = segs;
+    p.status = status;
+    return cuda_status(launch_kv_append(p, head_dim, n_segs, max_rows, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tf_status tf_attn_merge(const float *part_o, const float *part_m, const float *part_l, const uint8_t *part_flag,

@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, (D == 256) ? 1 : 2) attn_partial_ker
         w.pt_base = sg.pt_base;
         w.n_pg = sg.n_pages;
         const bool bad = w.q_row < 0 || w.n_rows < 0 || (int64_t)w.q_row + w.n_rows > p.n_rows_total ||
-                         w.n_keys < w.n_rows || w.pt_base < 0 || w.n_pg < 0 ||
+                         w.n_keys < (p.full ? (w.n_rows > 0 ? 1 : 0) : w.n_rows) || w.pt_base < 0 || w.n_pg < 0 ||
                          (int64_t)w.pt_base + w.n_pg > p.pt_len;
         if (bad) {
             if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, (D == 256) ? 1 : 2) attn_partial_ker
     w.key_lo = w.c * per;
     w.key_hi = min(w.n_keys, w.key_lo + per);
     const int i_min = w.q0 / p.group, i_max = (w.q0 + w.nq - 1) / p.group;
-    const int causal0 = w.n_keys - w.n_rows + 1;  // keys every row sees: [0, causal0)
+    // keys every row sees: [0, causal0) (with the full flag: all of them)
+    const int causal0 = p.full ? w.n_keys : w.n_keys - w.n_rows + 1;
     w.key_hi_eff = min(w.key_hi, causal0 + i_max);
     w.n_tiles = w.key_hi_eff > w.key_lo ? (w.key_hi_eff - w.key_lo + kTK - 1) / kTK : 0;
     const int full_hi = min(w.key_hi, causal0 + i_min);  // below this key no masking is needed

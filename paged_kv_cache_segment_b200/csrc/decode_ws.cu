@@ -98,7 +98,7 @@ __device__ __forceinline__ int ws_stream_splits(const WsParams &p, int s, uint32
     } else {
         const tf_seg e = p.segs[s];
         const bool bad = e.q_row < 0 || e.n_rows < 0 || (int64_t)e.q_row + e.n_rows > p.n_rows_total ||
-                         e.n_keys < e.n_rows || e.pt_base < 0 || e.n_pages < 0 ||
+                         e.n_keys < (p.full ? (e.n_rows > 0 ? 1 : 0) : e.n_rows) || e.pt_base < 0 || e.n_pages < 0 ||
                          (int64_t)e.pt_base + e.n_pages > p.pt_len;
         if (bad) {
             bits |= TF_DEV_BAD_SEG;
@@ -211,7 +211,9 @@ __device__ __forceinline__ WsItem ws_resolve(const WsParams &p, const int *prefi
         it.size = it.start = 0;
         it.wrap_at = 0x7fffffff;
     }
-    it.causal0 = it.n_keys - it.n_rows + 1;
+    // keys every row sees: [0, causal0); row i sees [0, causal0 + i) (with
+    // the full flag every row sees all n_keys)
+    it.causal0 = p.full ? it.n_keys : it.n_keys - it.n_rows + 1;
     it.full_hi = min(it.key_hi, it.causal0);
     return it;
 }

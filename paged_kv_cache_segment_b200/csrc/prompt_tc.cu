@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         n_pg = sg.n_pages;
         split = (int)blockIdx.x / p.n_qt;
         qt = p.n_qt - 1 - (int)blockIdx.x % p.n_qt;  // the most keys first
-        const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < T || pt_base < 0 ||
+        const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < (p.full ? (T > 0 ? 1 : 0) : T) || pt_base < 0 ||
                          n_pg < 0 || (int64_t)pt_base + n_pg > p.pt_len;
         if (bad) {
             if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
@@ -165,8 +165,10 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     }
     const int row0 = qt * RT;  // segment-relative first row
     const int rows_here = min(RT, T - row0);
-    const int key_hi_eff = min(key_hi_split, N - T + row0 + rows_here);  // keys the last valid row sees
-    const int full_hi = min(key_hi_eff, N - T + row0 + 1);               // keys every row of the tile sees
+    // row i of the segment sees keys [0, causal0 + i) (all N with the full flag)
+    const int causal0 = (PARTIAL && p.full) ? N : N - T + 1;
+    const int key_hi_eff = min(key_hi_split, causal0 + row0 + rows_here - 1);  // keys the last valid row sees
+    const int full_hi = min(key_hi_eff, causal0 + row0);                       // keys every row of the tile sees
     const int n_tiles = key_hi_eff > key_lo ? (key_hi_eff - key_lo + kBN - 1) / kBN : 0;
     if (PARTIAL && n_tiles == 0) {
         // no row of the tile sees a key of this split: m = -inf, l = 0, o = 0
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         const int qi = quad * 32 + lane;
         const int row_i = row0 + qi / G;  // chunk-relative
         const bool valid_row = row_i < T;
-        const int lim = valid_row ? (N - T + row_i + 1) : key_hi_eff;
+        const int lim = valid_row ? min(key_hi_eff, causal0 + row_i) : key_hi_eff;
         const float scale_log2 = p.scale_log2;
         float m_ref = -INFINITY, l_run = 0.f;
         uint32_t emax = 0, tail_bad = 0;

@@ -25,6 +25,7 @@ struct AttnParams {
     int64_t ring_slots_total;
     float scale_log2;  // scale * log2(e)
     int split_keys, n_splits_max, n_qgroups;
+    int full;  // every row sees all of its stream's keys (no causal count)
     // partial outputs [unit][n_splits_max](*D)
     float *part_o, *part_m, *part_l;
     uint8_t *part_flag;
@@ -61,8 +62,19 @@ struct PromptTcParams {
     // split-KV partials: segment table, splits, q-tiles of the grid, outputs
     const tf_seg *segs;
     int pt_len, split_keys, n_splits_max, n_qt;
+    int full;  // every row sees all of its stream's keys (no causal count)
     float *part_o, *part_m, *part_l;
     uint8_t *part_flag;
+    uint32_t *status;
+};
+
+// Parameters of the KV append (rows into their pages).
+struct AppendParams {
+    const uint16_t *k_rows, *v_rows;  // bf16 [n_rows_total][hkv][D]
+    uint16_t *k_pool, *v_pool;        // bf16 [n_pages][hkv][P][D]
+    int n_rows_total, hkv, n_pages, log2_page, pt_len;
+    const int32_t *page_table;
+    const tf_seg *segs;
     uint32_t *status;
 };
 
@@ -80,6 +92,7 @@ struct WsParams {
     int64_t ring_slots_total;
     float scale_log2;
     int split_keys, n_splits_max;
+    int full;  // every row sees all of its stream's keys (no causal count)
     float *part_o, *part_m, *part_l;
     uint8_t *part_flag;
     uint32_t *status;
@@ -101,6 +114,7 @@ bool prompt_tc_supported(int head_dim, int group, int page_size);
 bool decode_ws_supported(int head_dim, int n_segs);
 cudaError_t launch_decode_ws(const WsParams &p, int head_dim, bool ring, const void *k, const void *v,
                              int64_t n_items_bound, cudaStream_t st);
+cudaError_t launch_kv_append(const AppendParams &p, int head_dim, int n_segs, int max_rows, cudaStream_t st);
 cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, cudaStream_t st);
 bool partial_tc_supported(int head_dim, int group, int page_size, int split_keys);
 cudaError_t launch_partial_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, int n_segs,

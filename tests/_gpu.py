@@ -27,8 +27,9 @@ def status_word() -> torch.Tensor:
 
 
 def run_decode(b: wl.PagedBatch, *, split_keys=None, n_splits_max=None, host_tables=True, merge=True, segs=None,
-               page_table=None):
-    """Partials + merge for a paged batch.  Returns dict of numpy results."""
+               page_table=None, block=False):
+    """Partials + merge for a paged batch (block: every row over all of its
+    stream's keys).  Returns dict of numpy results."""
     split_keys = b.split_keys if split_keys is None else split_keys
     n_splits_max = b.n_splits_max if n_splits_max is None else n_splits_max
     segs = b.segs if segs is None else segs
@@ -41,7 +42,7 @@ def run_decode(b: wl.PagedBatch, *, split_keys=None, n_splits_max=None, host_tab
     pl = torch.full((rows, hq, n_splits_max), float("nan"), device=DEV)
     pf = torch.full((rows, hq, n_splits_max), 7, dtype=torch.uint8, device=DEV)
     st = status_word()
-    tf.tf_paged_attn_decode(q, kp, vp, pt, sg, scale=b.scale, split_keys=split_keys, n_splits_max=n_splits_max,
+    (tf.tf_paged_attn_block if block else tf.tf_paged_attn_decode)(q, kp, vp, pt, sg, scale=b.scale, split_keys=split_keys, n_splits_max=n_splits_max,
                             part_o=po, part_m=pm, part_l=pl, part_flag=pf, status=st,
                             segs_host=segs if host_tables else None,
                             page_table_host=page_table if host_tables else None)
