@@ -88,3 +88,37 @@ def test_host_checks_of_other_calls():
     seg = np.array([[0, 4, 3, 0, 1]], np.int32)  # more rows than keys
     assert lib.tf_paged_attn_prompt(FAKE, 4, 8, FAKE, FAKE, 4, 16, 2, 64, FAKE, 1, seg.ctypes.data_as(ctypes.c_void_p),
                                     0.1, FAKE, 1, None, FAKE, None) == 1
+
+
+def test_host_checks_of_block_and_append():
+    lib = tf.load()
+    segs = np.array([[0, 4, 2, 0, 1]], np.int32)  # a block of 4 rows over 2 keys
+    a = dict(q=FAKE, rows=4, hq=8, k=FAKE, v=FAKE, n_pages=16, psz=16, hkv=2, d=64, pt=FAKE, pt_len=8, segs=FAKE,
+             n_segs=1, segs_host=segs.ctypes.data_as(ctypes.c_void_p), pt_host=None, scale=0.125, split=16, nsm=2,
+             po=FAKE, pm=FAKE, pl=FAKE, pf=FAKE, st=FAKE, stream=None)
+    assert call_decode(**a) == 1  # the causal count needs a key per row
+    b = dict(a, d=96)
+    assert lib.tf_paged_attn_block(*b.values()) == 4  # unsupported head dim
+    none = segs.copy()
+    none[0, 2] = 0  # rows but no key at all
+    b = dict(a, segs_host=none.ctypes.data_as(ctypes.c_void_p))
+    assert lib.tf_paged_attn_block(*b.values()) == 1
+
+    def append(**kw):
+        c = dict(kr=FAKE, vr=FAKE, rows=4, kp=FAKE, vp=FAKE, n_pages=16, psz=16, hkv=2, d=64, pt=FAKE, pt_len=8,
+                 segs=FAKE, n_segs=1, segs_host=None, pt_host=None, st=FAKE, stream=None)
+        c.update(kw)
+        return lib.tf_kv_append(*c.values())
+
+    assert append(d=96) == 4
+    assert append(psz=24) == 4
+    assert append(kr=ctypes.c_void_p(0x10008)) == 6  # misaligned
+    assert append(n_segs=0) == 0
+    rows_past = np.array([[0, 2, 17, 0, 1]], np.int32)  # key 16 lies past the one page of 16
+    assert append(segs_host=rows_past.ctypes.data_as(ctypes.c_void_p)) == 2
+    few_keys = np.array([[0, 3, 2, 0, 1]], np.int32)  # more new rows than keys
+    assert append(segs_host=few_keys.ctypes.data_as(ctypes.c_void_p)) == 1
+    pt = np.array([16], np.int32)  # a page id outside the pool
+    ok = np.array([[0, 2, 5, 0, 1]], np.int32)
+    assert append(segs_host=ok.ctypes.data_as(ctypes.c_void_p), pt_host=pt.ctypes.data_as(ctypes.c_void_p),
+                  pt_len=1) == 3
