@@ -59,7 +59,8 @@ struct WsCfg {
     static constexpr int kPrefixMax = D == 256 ? 512 : 256;
     static constexpr int kMinBlocks = D == 256 ? 1 : 2;
     static constexpr int kQBytes = kWsQ * D * 2;
-    static constexpr int kCombBytes = (NC / 2) * kWsQ * D * 4;
+    static constexpr int kCombStride = D + 4;  // floats a query row of the combine buffer (no bank conflicts)
+    static constexpr int kCombBytes = (NC / 2) * kWsQ * kCombStride * 4;
     static constexpr int kOffQ = kStages * kStageBytes;
     static constexpr int kOffComb = kOffQ + kNQ * kQBytes;
     static constexpr int kOffPrefix = kOffComb + kCombBytes;
@@ -235,6 +236,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
     __shared__ __align__(8) uint64_t full_bar[C::kStages], empty_bar[C::kStages];
     __shared__ __align__(8) uint64_t qfull_bar[C::kNQ], qempty_bar[C::kNQ];
     __shared__ uint32_t s_meta[C::kStages];
+    __shared__ WsItem s_item[C::kNQ];  // the item of each query buffer, resolved by the producer
     __shared__ float comb_m[C::NC / 2][kWsQ], comb_l[C::NC / 2][kWsQ];
     __shared__ uint32_t comb_f[C::NC / 2][kWsQ];
     __shared__ int s_total, s_full;
@@ -403,6 +405,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                     break;
                 }
                 if (lane == 0) {
+                    s_item[qs] = it;  // published with the queries (the arrive below releases it)
                     const uint32_t qdst = sbase + C::kOffQ + qs * C::kQBytes;
                     const uint32_t qbytes = (uint32_t)(p.group * D * 2);
                     mbar_arrive_expect_tx(smem_u32(&qfull_bar[qs]), qbytes * it.n_rows);
@@ -495,15 +498,16 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
     const float scale_log2 = p.scale_log2;
     uint32_t tc = 0, qc = 0;
     for (int k = 0, L = ws_snake(0, bid, grid); L < total; L = ws_snake(++k, bid, grid)) {
-        const WsItem it = ws_resolve<RING>(p, prefix, prefix_full, tail_order, n_full, L);
-        const int q_item = it.n_rows * p.group;
-        // queries of this item -> B fragments (Q^T), kept in registers
+        // the item (resolved by the producer) and its queries -> B fragments
+        // (Q^T), kept in registers
         const uint32_t qs = qc % C::kNQ;
         const bool q_ok = mbar_wait(smem_u32(&qfull_bar[qs]), (qc / C::kNQ) & 1);
         if (named_bar_red_or(1, C::NC * 32, !q_ok)) {  // every consumer warp leaves together
             if (tid == 0) atomicOr(p.status, TF_DEV_TIMEOUT);
             break;
         }
+        const WsItem it = s_item[qs];
+        const int q_item = it.n_rows * p.group;
         uint32_t qb[D / 16][2];
         {
             const uint32_t qsrc = sbase + C::kOffQ + qs * C::kQBytes;
@@ -691,13 +695,13 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
         }
         uint32_t f0 = (e0 == 0x7f800000u) | tb0 | badp, f1 = (e1 == 0x7f800000u) | tb1 | badp;
         auto put = [&](int slot) {
-            float *dst = comb_o + slot * kWsQ * D;
+            float *dst = comb_o + slot * kWsQ * C::kCombStride;
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt) {
-                dst[qa * D + 16 * mt + gq] = o[mt][0];
-                dst[qb_ * D + 16 * mt + gq] = o[mt][1];
-                dst[qa * D + 16 * mt + gq + 8] = o[mt][2];
-                dst[qb_ * D + 16 * mt + gq + 8] = o[mt][3];
+                dst[qa * C::kCombStride + 16 * mt + gq] = o[mt][0];
+                dst[qb_ * C::kCombStride + 16 * mt + gq] = o[mt][1];
+                dst[qa * C::kCombStride + 16 * mt + gq + 8] = o[mt][2];
+                dst[qb_ * C::kCombStride + 16 * mt + gq + 8] = o[mt][3];
             }
             if (gq == 0) {
                 comb_m[slot][qa] = m0;
@@ -709,7 +713,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             }
         };
         auto take = [&](int slot) {
-            const float *src = comb_o + slot * kWsQ * D;
+            const float *src = comb_o + slot * kWsQ * C::kCombStride;
             const float ma = comb_m[slot][qa], mb = comb_m[slot][qb_];
             const float la = comb_l[slot][qa], lb = comb_l[slot][qb_];
             f0 |= comb_f[slot][qa];
@@ -723,10 +727,10 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             m1 = M1;
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt) {
-                o[mt][0] = o[mt][0] * w0 + src[qa * D + 16 * mt + gq] * wa;
-                o[mt][1] = o[mt][1] * w1 + src[qb_ * D + 16 * mt + gq] * wb;
-                o[mt][2] = o[mt][2] * w0 + src[qa * D + 16 * mt + gq + 8] * wa;
-                o[mt][3] = o[mt][3] * w1 + src[qb_ * D + 16 * mt + gq + 8] * wb;
+                o[mt][0] = o[mt][0] * w0 + src[qa * C::kCombStride + 16 * mt + gq] * wa;
+                o[mt][1] = o[mt][1] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq] * wb;
+                o[mt][2] = o[mt][2] * w0 + src[qa * C::kCombStride + 16 * mt + gq + 8] * wa;
+                o[mt][3] = o[mt][3] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq + 8] * wb;
             }
         };
         named_bar_sync(1, C::NC * 32);  // the previous item's readers are done with comb
@@ -764,7 +768,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                                    : (int64_t)(it.q_row + i) * p.hq + it.g * p.group + hl;
             const int64_t at = u * p.n_splits_max + it.c;
             *reinterpret_cast<float4 *>(p.part_o + at * D + d4) =
-                *reinterpret_cast<const float4 *>(comb_o + qq * D + d4);
+                *reinterpret_cast<const float4 *>(comb_o + qq * C::kCombStride + d4);
             if (d4 == 0) {
                 const float mm = comb_m[0][qq];
                 p.part_m[at] = (mm == -INFINITY) ? -INFINITY : mm * kLn2;
