@@ -6,8 +6,10 @@
 // flagged.  Readings: values compare as real numbers (-0 == +0), a flagged
 // row reports id -1.
 //
-// Each row is split over a cluster of 8 CTAs.  Every thread loads its share
-// with 16-byte loads (eight in flight) and works on 32-bit words, two bf16
+// Each row is split over a cluster of two CTAs of 1,024 threads (a 128,000-
+// wide row is then one batch of eight 16-byte loads a thread, all in flight,
+// with the fewest CTAs to launch and barriers to cross).  Every thread works
+// on 32-bit words, two bf16
 // values each: max.bf16x2 keeps the largest value of each half and
 // max.u16x2 over the magnitude bits keeps the largest exponent pattern
 // (reaching 0x7f80 means a NaN or an infinity).  The cluster agrees on the
@@ -33,7 +35,7 @@ namespace cg = cooperative_groups;
 
 namespace tfp {
 
-constexpr int kArgThreads = 256;
+constexpr int kArgThreads = 1024;
 constexpr int kArgBatch = 8;  // 16-byte vectors in flight per thread
 constexpr int kArgWarps = kArgThreads / 32;
 

@@ -120,6 +120,6 @@ bool partial_tc_supported(int head_dim, int group, int page_size, int split_keys
 cudaError_t launch_partial_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, int n_segs,
                               cudaStream_t st);
 
-constexpr int kArgmaxCluster = 8;
+constexpr int kArgmaxCluster = 2;
 
 }  // namespace tfp
