@@ -431,6 +431,20 @@ def bench_verify(wl, dev, steps, peaks, traffic):
         run.merge(k)
         run.argmax(k)
     per, total = timed_steps([run.partial, run.merge, run.argmax], steps)
+
+    # the same round as one call (tf_verify_round): merge and argmax launch as
+    # programmatic dependents, timed at the round's ends
+    import paged_kv_cache_segment_b200 as tf
+
+    def round_call(k):
+        x = run.sets[k % len(run.sets)]
+        tf.tf_verify_round(x["q"], x["kp"], x["vp"], x["pt"], x["segs"], scale=b.scale, split_keys=b.split_keys,
+                           n_splits_max=b.n_splits_max, part_o=run.po, part_m=run.pm, part_l=run.pl,
+                           part_flag=run.pf, out=run.out, flags=run.fl, status=run.st, logits=x["logits"],
+                           ids=run.ids, id_flags=run.afl, segs_host=b.segs)
+
+    round_call(0)
+    _, round_total = timed_steps([round_call], steps)
     kv = b.kv_bytes()
     pms, mms, ams = per[0] / steps, per[1] / steps, per[2] / steps
     flops = 4 * b.head_dim * sum(int(s[1]) * b.n_q_heads * (int(s[2]) - int(s[1]) + 1) + b.n_q_heads *
@@ -445,6 +459,10 @@ def bench_verify(wl, dev, steps, peaks, traffic):
                                              traffic.get("prompt_tc:shared_verify")),
                                     kernel="prompt_tc_kernel<256, hilo, partial>"),
                    "launches": 2 * steps, "l2": "8 rotating copies"},
+        "round": {"workload": "the shared verify round in one call: partials, merge, argmax of its 62 rows",
+                  "ms": round(round_total / steps, 5), "ms_three_calls": round(total / steps, 5),
+                  "kv_plus_logit_gbs": round((kv + arg_bytes) / (round_total / steps) / 1e6, 2),
+                  "launches": 3 * steps},
         "argmax": {"workload": f"{rows} rows x 128,000 bf16 ~N(0,3), ties in ~1/4 of rows",
                    "rows_per_s": round(rows / (ams * 1e-3), 1), "ms": round(ams, 5),
                    "roofline": roofline("hbm", arg_bytes / (ams * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",

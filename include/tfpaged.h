@@ -162,6 +162,36 @@ TF_API tf_status tf_paged_attn_block(const void *q, int32_t n_rows_total, int32_
                               uint8_t *part_flag, uint32_t *status, tf_stream_t stream);
 
 /*
+ * One verify round's device work in one call: split-KV partials of every
+ * stream (the causal count, or with `full` != 0 the FULL rule of
+ * tf_paged_attn_block), their merge into out/flags, then the greedy argmax of
+ * n_logit_rows logit rows into ids/id_flags.  The merge and the argmax are
+ * launched as programmatic dependents of the launch before each, so their
+ * launches overlap the previous kernel's tail; each still reads its inputs
+ * only after the previous grid has finished.  Sources: #1394 ("lfm2: a
+ * cheaper DSpark hold", commit list: a hold's attention partials take all of
+ * its query rows in one wave, then merge in one, with a barrier only where a
+ * step reads an earlier step's writes) and #1503 (commit list: the verify
+ * rows' argmax on the GPU instead of a host scan).
+ *
+ * Arguments: those of tf_paged_attn_decode, tf_attn_merge (out, flags) and
+ * tf_argmax_rows (logits bf16 [n_logit_rows][ld], n_cols, ids, id_flags);
+ * n_logit_rows = 0 skips the argmax.  The logits are the caller's (the rows'
+ * head outputs); nothing in the attention feeds them.  Every argument is
+ * checked before the first launch; the result equals the three calls made
+ * one after another.
+ */
+TF_API tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                                 const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                                 int32_t head_dim, const int32_t *page_table, int32_t page_table_len,
+                                 const tf_seg *segs, int32_t n_segs, const tf_seg *segs_host,
+                                 const int32_t *page_table_host, float scale, int32_t split_keys,
+                                 int32_t n_splits_max, int32_t full, float *part_o, float *part_m, float *part_l,
+                                 uint8_t *part_flag, float *out, uint8_t *flags, const void *logits,
+                                 int32_t n_logit_rows, int32_t n_cols, int64_t ld, int32_t *ids, uint8_t *id_flags,
+                                 uint32_t *status, tf_stream_t stream);
+
+/*
  * Append each stream's new rows' keys and values into its pages: the
  * counterpart of tf_wrows_put in #1653 ("spark25 CUDA: the full layers'
  * caches in pages of the core pool", PR body: the rows kernel writes kr/vr

@@ -22,4 +22,5 @@ from .binding import (  # noqa: F401
     tf_ring_attn_noalloc,
     tf_ring_workspace_bytes,
     tf_status_str,
+    tf_verify_round,
 )

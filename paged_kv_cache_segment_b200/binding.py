@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "TF_OK", 1: "TF_ERR_ARG", 2: "TF_ERR_PAST_PAGES", 3: "TF_ERR_
 TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS = 1, 2, 4, 8
 TF_OUT_F32, TF_OUT_BF16 = 0, 1
 
-EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
+EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
            "tf_ring_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_status_str", "tf_abi_version")
 # bytes of the scratch array tf_ring_attn_noalloc keeps in the library's device image
 TF_RING_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -57,6 +57,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                          P, P, P, P, P, P]
     lib.tf_paged_attn_block.argtypes = lib.tf_paged_attn_decode.argtypes
     lib.tf_kv_append.argtypes = [P, P, i32, P, P, i32, i32, i32, i32, P, i32, P, i32, P, P, P, P]
+    lib.tf_verify_round.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, i32, P, P, f32, i32, i32, i32,
+                                    P, P, P, P, P, P, P, i32, i32, i64, P, P, P, P]
     lib.tf_attn_merge.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P]
     lib.tf_paged_attn_prompt.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, f32, P, i32, P, P, P]
     lib.tf_ring_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, f32, i32, i32, P, sz, P, P, P, P]
@@ -67,7 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_status_str.argtypes = [ctypes.c_int]
     lib.tf_status_str.restype = ctypes.c_char_p
     lib.tf_abi_version.restype = ctypes.c_int32
-    for name in ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
+    for name in ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
                  "tf_ring_attn_noalloc", "tf_argmax_rows"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -181,6 +183,37 @@ def tf_kv_append(k_rows, v_rows, k_pool, v_pool, page_table, segs, *, status, se
         page_table.numel(), _dev(segs, "segs", (torch.int32,)), segs.numel() // 5, _host_ptr(sh), _host_ptr(pth),
         _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
     _check("tf_kv_append", rc)
+
+
+def tf_verify_round(q, k_pool, v_pool, page_table, segs, *, scale, split_keys, n_splits_max, part_o, part_m, part_l,
+                    part_flag, out, flags, status, logits=None, ids=None, id_flags=None, n_cols=None, full=False,
+                    segs_host=None, page_table_host=None, stream=None):
+    """Partials, merge and (when logits are given) the row argmax of one round in one call (tf_verify_round)."""
+    lib = load()
+    rows, hq, d = q.shape
+    n_pages, hkv, psz, d2 = k_pool.shape
+    if d2 != d or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("q / pool head dims disagree")
+    sh = as_segs_np(segs_host) if segs_host is not None else None
+    pth = np.ascontiguousarray(np.asarray(page_table_host, np.int32)) if page_table_host is not None else None
+    if logits is not None:
+        if logits.dim() != 2 or logits.stride(1) != 1:
+            raise ValueError("logits must be 2-D with unit column stride")
+        n_lr, ld = logits.shape[0], logits.stride(0)
+        nc = logits.shape[1] if n_cols is None else int(n_cols)
+        lp, ip, fp = _dev(logits, "logits", BF16), _dev(ids, "ids", (torch.int32,)), _dev(id_flags, "id_flags",
+                                                                                         (torch.uint8,))
+    else:
+        n_lr, ld, nc, lp, ip, fp = 0, 0, 0, None, None, None
+    rc = lib.tf_verify_round(
+        _dev(q, "q", BF16), rows, hq, _dev(k_pool, "k_pool", BF16), _dev(v_pool, "v_pool", BF16), n_pages, psz, hkv, d,
+        _dev(page_table, "page_table", (torch.int32,)), page_table.numel(), _dev(segs, "segs", (torch.int32,)),
+        segs.numel() // 5, _host_ptr(sh), _host_ptr(pth), float(scale), int(split_keys), int(n_splits_max),
+        int(bool(full)), _dev(part_o, "part_o", (torch.float32,)), _dev(part_m, "part_m", (torch.float32,)),
+        _dev(part_l, "part_l", (torch.float32,)), _dev(part_flag, "part_flag", (torch.uint8,)),
+        _dev(out, "out", (torch.float32,)), _dev(flags, "flags", (torch.uint8,)), lp, n_lr, nc, ld, ip, fp,
+        _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
+    _check("tf_verify_round", rc)
 
 
 def tf_attn_merge(part_o, part_m, part_l, part_flag, out, flags, *, stream=None):

@@ -274,6 +274,36 @@ tf_status tf_kv_append(const void *k_rows, const void *v_rows, int32_t n_rows_to
     return cuda_status(launch_kv_append(p, head_dim, n_segs, max_rows, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
+                          const void *v_pool, int32_t n_pages, int32_t page_size, int32_t n_kv_heads,
+                          int32_t head_dim, const int32_t *page_table, int32_t page_table_len, const tf_seg *segs,
+                          int32_t n_segs, const tf_seg *segs_host, const int32_t *page_table_host, float scale,
+                          int32_t split_keys, int32_t n_splits_max, int32_t full, float *part_o, float *part_m,
+                          float *part_l, uint8_t *part_flag, float *out, uint8_t *flags, const void *logits,
+                          int32_t n_logit_rows, int32_t n_cols, int64_t ld, int32_t *ids, uint8_t *id_flags,
+                          uint32_t *status, tf_stream_t stream) {
+    // the argmax's arguments first, so a refusal launches nothing
+    if (n_logit_rows < 0) return TF_ERR_ARG;
+    if (n_logit_rows > 0) {
+        if (n_cols <= 0 || ld < n_cols || !logits || !ids || !id_flags) return TF_ERR_ARG;
+        if ((reinterpret_cast<uintptr_t>(logits) & 1u) != 0) return TF_ERR_ALIGN;
+    }
+    if (n_rows_total > 0 && n_q_heads > 0 && (!out || !flags)) return TF_ERR_ARG;
+    if (n_rows_total > 0 && out && !aligned16(out)) return TF_ERR_ALIGN;
+    tf_status st = paged_partials(full != 0, q, n_rows_total, n_q_heads, k_pool, v_pool, n_pages, page_size,
+                                  n_kv_heads, head_dim, page_table, page_table_len, segs, n_segs, segs_host,
+                                  page_table_host, scale, split_keys, n_splits_max, part_o, part_m, part_l,
+                                  part_flag, status, stream);
+    if (st != TF_OK) return st;
+    if (n_segs > 0 && n_rows_total > 0) {
+        st = tf_attn_merge(part_o, part_m, part_l, part_flag, n_rows_total, n_q_heads, head_dim, n_splits_max, out,
+                           flags, stream);
+        if (st != TF_OK) return st;
+    }
+    if (n_logit_rows == 0) return TF_OK;
+    return tf_argmax_rows(logits, n_logit_rows, n_cols, ld, ids, id_flags, stream);
+}
+
 tf_status tf_attn_merge(const float *part_o, const float *part_m, const float *part_l, const uint8_t *part_flag,
                         int32_t n_rows_total, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max, float *out,
                         uint8_t *flags, tf_stream_t stream) {

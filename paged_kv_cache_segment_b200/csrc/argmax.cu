@@ -61,6 +61,9 @@ __device__ __forceinline__ uint32_t unkey16(uint32_t k) { return (k & 0x8000u) ?
 
 template <bool VEC>
 __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThreads) argmax_kernel(const ArgmaxParams p) {
+    // may run as a programmatic dependent of the launch before it (a verify
+    // round's merge): nothing is read before that grid has finished
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -190,12 +193,17 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
 
 cudaError_t launch_argmax(const ArgmaxParams &p, bool vec, cudaStream_t st) {
     if (p.n_rows == 0) return cudaSuccess;
-    const dim3 grid(kArgmaxCluster, (unsigned)(p.n_rows < 65535 ? p.n_rows : 65535));
-    if (vec)
-        argmax_kernel<true><<<grid, kArgThreads, 0, st>>>(p);
-    else
-        argmax_kernel<false><<<grid, kArgThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(kArgmaxCluster, (unsigned)(p.n_rows < 65535 ? p.n_rows : 65535));
+    cfg.blockDim = dim3(kArgThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return vec ? cudaLaunchKernelEx(&cfg, argmax_kernel<true>, p) : cudaLaunchKernelEx(&cfg, argmax_kernel<false>, p);
 }
 
 }  // namespace tfp

@@ -572,6 +572,9 @@ __global__ void __launch_bounds__(kThreads, (D == 256) ? 1 : 2) attn_partial_ker
 template <int D, bool RING>
 __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // a dependent launch (a verify round's argmax) may start; it waits for
+    // this grid's completion before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t u = (int64_t)blockIdx.x * 4 + warp;
     if (u >= p.n_units) return;

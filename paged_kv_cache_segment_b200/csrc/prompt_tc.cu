@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     __shared__ uint32_t s_xbad[2][2][kQM];  // [exchange][column half][row]: nonfinite findings
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the merge that follows may launch now; it waits for this grid to finish
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     unsigned char *sbase_ptr = smem_raw + (sbase - smem_u32(smem_raw));
     auto sK = [&](int s) { return sbase + C::kOffK + s * C::kKVBytes; };
