@@ -364,11 +364,11 @@ def run_native(args):
         if want(args, "ring"):
             sec["ring"] = bench_ring(wl, tf, dev, ks, peaks, traffic)
         if want(args, "prompt"):
-            sec["prompt"] = bench_prompt(wl, tf, dev, max(3, ks // 4), peaks)
+            sec["prompt"] = bench_prompt(wl, tf, dev, max(3, ks // 4), peaks, traffic)
         if want(args, "block"):
-            sec["block"] = bench_block(wl, tf, dev, ks, peaks)
+            sec["block"] = bench_block(wl, tf, dev, ks, peaks, traffic)
         if want(args, "append"):
-            sec["append"] = bench_append(wl, tf, dev, ks, peaks)
+            sec["append"] = bench_append(wl, tf, dev, ks, peaks, traffic)
         result["secondary"] = sec
         result["gpu_launches_secondary"] = sum(v.get("launches", 0) for v in sec.values())
     if rank == 0 and world == 1 and want(args, "cpu"):
@@ -507,7 +507,7 @@ def bench_ring(wl, tf, dev, steps, peaks, traffic):
             "l2": "3 rotating copies"}
 
 
-def bench_prompt(wl, tf, dev, steps, peaks):
+def bench_prompt(wl, tf, dev, steps, peaks, traffic):
     import torch
 
     b, spans = wl.long_prompt(4)
@@ -535,11 +535,14 @@ def bench_prompt(wl, tf, dev, steps, peaks):
     return {"workload": "long causal prompt: 15,000 tokens in 2,048-row chunks, 16/4 heads, D256, P32, 469 shuffled "
                         "pages, bf16 out", "tflops": round(tfl, 2), "ms_per_step": round(ms, 4),
             "algorithmic_flops": flops,
-            "roofline": roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s"), "launches": len(segs) * steps,
+            "roofline": dict(roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s",
+                                      traffic.get("prompt_tc:long_prompt")), kernel="prompt_tc_kernel<256, bf16>",
+                             traffic_is="DRAM bytes per chunk launch (mean of 8); the K/V of a chunk is re-read from L2"),
+            "launches": len(segs) * steps,
             "l2": "2 rotating copies"}
 
 
-def bench_block(wl, tf, dev, steps, peaks):
+def bench_block(wl, tf, dev, steps, peaks, traffic):
     """A drafter-block round: 16 streams, each a block of 9 rows seeing all of
     its stream's keys (the FULL rule), contexts U{1,024..8,192}, 32/8 heads,
     D 128, pages of 32, 512-key partials + merge; 3 rotating copies."""
@@ -566,12 +569,13 @@ def bench_block(wl, tf, dev, steps, peaks):
     return {"workload": "drafter blocks: 16 streams x 9 rows, every row over all its stream's keys, contexts "
                         "U{1024..8192}, 32/8 heads, D128, P32, 512-key partials + merge",
             "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2), "ms_per_step": round(ms, 5),
-            "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"),
+            "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                                      traffic.get("prompt_tc:drafter_block")),
                              kernel="prompt_tc_kernel<128, hilo, partial> + merge (the whole step)"),
             "launches": 2 * steps, "l2": "3 rotating copies"}
 
 
-def bench_append(wl, tf, dev, steps, peaks):
+def bench_append(wl, tf, dev, steps, peaks, traffic):
     """The 15,000-token prompt's keys and values appended in one call (4
     kv-heads, D 256, pages of 32) into a shuffled pool; 3 rotating pool
     copies.  Bytes: every row read once from the row arrays and written once
@@ -606,7 +610,8 @@ def bench_append(wl, tf, dev, steps, peaks):
     gbs = moved / (ms * 1e-3) / 1e9
     return {"workload": "append the 15,000-token prompt's K/V rows into 469 shuffled pages of 32 in one call "
                         "(4 kv-heads, D256)", "gbs": round(gbs, 2), "ms_per_step": round(ms, 5),
-            "bytes_per_step": moved, "roofline": dict(roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
+            "bytes_per_step": moved, "roofline": dict(roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s",
+                                                               traffic.get("kv_append:long_prompt")),
                                                       kernel="kv_append_kernel<256>"),
             "launches": len(calls) * steps, "l2": "3 rotating pool copies (rows arrays resident)"}
 
