@@ -117,7 +117,11 @@ __global__ void __launch_bounds__(kPTThreads, 1)
     volatile uint32_t *abort_flag = &s_abort;
 
     const int G = p.group, RT = kQM / p.group;  // rows a tile
-    const int g = blockIdx.y;
+    // partials: kv-head blockIdx.y; a prompt chunk: the launch order (block
+    // x fastest, then y) walks the query tiles from the most keys down, every
+    // kv-head's tile in turn, so the longest tiles of all heads start first
+    const int lin = (int)(blockIdx.y * gridDim.x + blockIdx.x);
+    const int g = PARTIAL ? (int)blockIdx.y : lin % (int)gridDim.y;
     const int P = 1 << p.log2_page, BR = P < kBN ? P : kBN, n_box = kBN / BR;
 
     // ---- the work item: a segment (the prompt's one, or entry blockIdx.z of
@@ -162,7 +166,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         key_lo = split * p.split_keys;
         key_hi_split = min(N, key_lo + p.split_keys);
     } else {
-        qt = (int)gridDim.x - 1 - (int)blockIdx.x;  // the most keys first
+        qt = (int)gridDim.x - 1 - lin / (int)gridDim.y;  // the most keys first
         key_hi_split = N;
     }
     const int row0 = qt * RT;  // segment-relative first row
