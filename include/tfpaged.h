@@ -245,6 +245,14 @@ TF_API tf_status tf_attn_merge(const float *part_o, const float *part_m, const f
  *
  *  seg_host  the stream's segment, in HOST memory (the chunk's size sets the grid)
  *
+ * Ordering: the chunk may begin while the call before it on the stream is
+ * still finishing, when that call is one of this library's attention or
+ * merge calls (consecutive chunks overlap, the next filling the SMs the last
+ * one's final wave leaves idle).  It reads only q, the pools and the page
+ * table, which those calls never write; two such calls must not write the
+ * same out rows.  After any other work on the stream (a kernel of the
+ * caller's, tf_kv_append, a copy) it starts when that work has finished.
+ *
  * Supported: head_dim in {64, 128, 256}; page sizes as for decode.
  */
 TF_API tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,

@@ -619,8 +619,26 @@ static cudaError_t launch_tc_t(const PromptTcParams &p, const void *k, const voi
     if (e != cudaSuccess) return e;
     const dim3 grid = PARTIAL ? dim3((unsigned)(p.n_qt * p.n_splits_max), (unsigned)p.hkv, (unsigned)n_segs)
                               : dim3((unsigned)((p.n_rows + RT - 1) / RT), (unsigned)p.hkv);
-    kern<<<grid, kPTThreads, PTCfg<D>::kSmemBytes, st>>>(mk, mv, p);
-    return cudaGetLastError();
+    if (PARTIAL) {
+        kern<<<grid, kPTThreads, PTCfg<D>::kSmemBytes, st>>>(mk, mv, p);
+        return cudaGetLastError();
+    }
+    // A prompt chunk may start while the call before it on the stream (this
+    // library's previous chunk, or another of its attention calls) finishes:
+    // it reads q, the pools and the page table, which none of them writes, so
+    // the next chunk's tiles fill the SMs the previous chunk's last wave
+    // leaves idle.
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kPTThreads);
+    cfg.dynamicSmemBytes = PTCfg<D>::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
 }
 
 cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, cudaStream_t st) {
