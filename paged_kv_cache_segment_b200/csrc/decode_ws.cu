@@ -501,12 +501,12 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
         // the item (resolved by the producer) and its queries -> B fragments
         // (Q^T), kept in registers
         const uint32_t qs = qc % C::kNQ;
+        // (no barrier here: a warp that finishes an item's combine late joins
+        // the next item late; a wait that gives up skips the item's tiles and
+        // the loop-end barrier takes every warp out)
         const bool q_ok = mbar_wait(smem_u32(&qfull_bar[qs]), (qc / C::kNQ) & 1);
-        if (named_bar_red_or(1, C::NC * 32, !q_ok)) {  // every consumer warp leaves together
-            if (tid == 0) atomicOr(p.status, TF_DEV_TIMEOUT);
-            break;
-        }
-        const WsItem it = s_item[qs];
+        WsItem it = s_item[qs];
+        if (!q_ok) it.key_lo = it.key_hi = 0;
         const int q_item = it.n_rows * p.group;
         uint32_t qb[D / 16][2];
         {
@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
         uint32_t e0 = 0, e1 = 0, tb0 = 0, tb1 = 0, badp = 0;
         const int kb = warp * 16;
-        bool aborted = false;
+        bool aborted = !q_ok;
 
         for (int j0 = it.key_lo; j0 < it.key_hi;) {
             const int rows = ws_tile_rows<C::TK>(it, j0);
@@ -733,15 +733,20 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                 o[mt][3] = o[mt][3] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq + 8] * wb;
             }
         };
-        named_bar_sync(1, C::NC * 32);  // the previous item's readers are done with comb
-#pragma unroll
-        for (int half = C::NC / 2; half >= 1; half >>= 1) {
-            if (warp >= half && warp < 2 * half) put(warp - half);
-            named_bar_sync(1, C::NC * 32);
-            if (warp < half) take(warp);
-            named_bar_sync(1, C::NC * 32);
+        // Warps 2 and 3 hand their states to warps 0 and 1 and go on to the
+        // next item; warp 1 then hands its state to warp 0, which writes the
+        // item's partials from its registers.  The slots are free again before
+        // the next item's combine: every warp passes the loop-end barrier first.
+        if (warp >= 2) put(warp - 2);
+        named_bar_sync(1, C::NC * 32);
+        if (warp < 2) {
+            take(warp);
+            named_bar_sync(2, 64);  // warp 0 has read slot 0: warp 1 may refill it
+            if (warp == 1) put(0);
+            named_bar_sync(2, 64);
         }
         if (warp == 0) {
+            take(0);
             bool nf0 = !isfinite(l0), nf1 = !isfinite(l1);
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt) {
@@ -755,25 +760,41 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             }
             f0 |= nf0;
             f1 |= nf1;
-            __syncwarp();
-            put(0);
-        }
-        named_bar_sync(1, C::NC * 32);
-        // write the partials of the item's real queries, coalesced over D
-        const int ctid = tid;  // 0 .. NC*32-1
-        for (int idx = ctid; idx < q_item * (D / 4); idx += C::NC * 32) {
-            const int qq = idx / (D / 4), d4 = (idx % (D / 4)) * 4;
-            const int i = qq / p.group, hl = qq - i * p.group;
-            const int64_t u = RING ? (int64_t)it.s * p.hq + it.g * p.group + hl
-                                   : (int64_t)(it.q_row + i) * p.hq + it.g * p.group + hl;
-            const int64_t at = u * p.n_splits_max + it.c;
-            *reinterpret_cast<float4 *>(p.part_o + at * D + d4) =
-                *reinterpret_cast<const float4 *>(comb_o + qq * C::kCombStride + d4);
-            if (d4 == 0) {
-                const float mm = comb_m[0][qq];
-                p.part_m[at] = (mm == -INFINITY) ? -INFINITY : mm * kLn2;
-                p.part_l[at] = comb_l[0][qq];
-                p.part_flag[at] = (uint8_t)(comb_f[0][qq] ? 1 : 0);
+            // this lane's queries qa, qb_ and dims 16 mt + gq (+ 8): eight
+            // consecutive floats of a row per four lanes
+            auto slot_of = [&](int qq) {
+                const int i = qq / p.group, hl = qq - i * p.group;
+                const int64_t u = RING ? (int64_t)it.s * p.hq + it.g * p.group + hl
+                                       : (int64_t)(it.q_row + i) * p.hq + it.g * p.group + hl;
+                return u * p.n_splits_max + it.c;
+            };
+            if (qa < q_item) {
+                const int64_t at = slot_of(qa);
+                float *dst = p.part_o + at * D;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    dst[16 * mt + gq] = o[mt][0];
+                    dst[16 * mt + gq + 8] = o[mt][2];
+                }
+                if (gq == 0) {
+                    p.part_m[at] = (m0 == -INFINITY) ? -INFINITY : m0 * kLn2;
+                    p.part_l[at] = l0;
+                    p.part_flag[at] = (uint8_t)(f0 ? 1 : 0);
+                }
+            }
+            if (qb_ < q_item) {
+                const int64_t at = slot_of(qb_);
+                float *dst = p.part_o + at * D;
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    dst[16 * mt + gq] = o[mt][1];
+                    dst[16 * mt + gq + 8] = o[mt][3];
+                }
+                if (gq == 0) {
+                    p.part_m[at] = (m1 == -INFINITY) ? -INFINITY : m1 * kLn2;
+                    p.part_l[at] = l1;
+                    p.part_flag[at] = (uint8_t)(f1 ? 1 : 0);
+                }
             }
         }
     }
