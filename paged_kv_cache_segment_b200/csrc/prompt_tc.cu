@@ -287,16 +287,12 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             __syncwarp();
         };
         if (n_tiles > 0 && wwait(bar(kBarQ), 0) && wwait(bar(kBarKFull), 0)) issue_qk(0);
-        for (int j = 0; j < n_tiles; ++j) {
+        // every lane tests, the warp acts on the answer all lanes agree on
+        auto ready = [&](uint32_t bb, uint32_t phase) { return __all_sync(0xffffffffu, mbar_test_wait(bb, phase)); };
+        // O += P(j) V(j)
+        auto issue_pv = [&](int j) {
             const int b = j & 1, s = j % kKVStages;
-            // the next tile's scores while the softmax warps work on this one;
-            // its S buffer held P(j-1), whose P V was issued before (in order)
-            const int j1 = j + 1;
-            if (j1 < n_tiles && wwait(bar(kBarKFull + j1 % kKVStages), (uint32_t)((j1 / kKVStages) & 1))) issue_qk(j1);
-            // P(j) written (and V(j) cleaned) and V(j) landed: O += P V
-            const bool ok = wwait(bar(kBarPr + b), (uint32_t)((j >> 1) & 1)) &&
-                            wwait(bar(kBarVFull + s), (uint32_t)((j / kKVStages) & 1));
-            if (ok && lane == 0) {
+            if (lane == 0) {
                 tc_fence_after();
                 const uint32_t sb = tmem + (b ? kColS1 : kColS0);
 #pragma unroll
@@ -309,6 +305,39 @@ __global__ void __launch_bounds__(kPTThreads, 1)
                 umma_commit(bar(kBarVFree + s));
             }
             __syncwarp();
+        };
+        for (int j = 0; j < n_tiles && !*abort_flag; ++j) {
+            const int b = j & 1, s = j % kKVStages, j1 = j + 1;
+            // Two independent groups: the next tile's scores QK(j+1) (its S
+            // buffer held P(j-1), whose P V went out before, in order) and
+            // P V(j) (P written, V landed and cleaned).  They touch different
+            // S buffers, so whichever is ready goes out first.  The poll is
+            // bounded like every wait; P V(j+1) and QK(j+2) come only after both.
+            bool need_qk = j1 < n_tiles, need_pv = true;
+            const uint64_t t_poll = global_ns();
+            while (need_qk || need_pv) {
+                bool moved = false;
+                if (need_qk && ready(bar(kBarKFull + j1 % kKVStages), (uint32_t)((j1 / kKVStages) & 1))) {
+                    issue_qk(j1);
+                    need_qk = false;
+                    moved = true;
+                }
+                if (need_pv && ready(bar(kBarPr + b), (uint32_t)((j >> 1) & 1)) &&
+                    ready(bar(kBarVFull + s), (uint32_t)((j / kKVStages) & 1))) {
+                    issue_pv(j);
+                    need_pv = false;
+                    moved = true;
+                }
+                if (!moved) {
+                    const bool give_up = __any_sync(0xffffffffu, *abort_flag != 0 ||
+                                                                   global_ns() - t_poll > 2000000000ull);
+                    if (give_up) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
         }
     } else {
         // ================= softmax warps: row qi of the tile, key columns 32h .. 32h + 31
