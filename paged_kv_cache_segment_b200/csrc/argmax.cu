@@ -60,7 +60,8 @@ __device__ __forceinline__ uint32_t key16(uint32_t b) { return (b & 0x8000u) ? (
 __device__ __forceinline__ uint32_t unkey16(uint32_t k) { return (k & 0x8000u) ? (k ^ 0x8000u) : (k ^ 0xffffu); }
 
 template <bool VEC>
-__global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThreads) argmax_kernel(const ArgmaxParams p) {
+__global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThreads)
+    argmax_kernel(const ArgmaxParams p) {
     // may run as a programmatic dependent of the launch before it (a verify
     // round's merge): nothing is read before that grid has finished
     asm volatile("griddepcontrol.wait;" ::: "memory");

@@ -137,8 +137,9 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         n_pg = sg.n_pages;
         split = (int)blockIdx.x / p.n_qt;
         qt = p.n_qt - 1 - (int)blockIdx.x % p.n_qt;  // the most keys first
-        const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < (p.full ? (T > 0 ? 1 : 0) : T) || pt_base < 0 ||
-                         n_pg < 0 || (int64_t)pt_base + n_pg > p.pt_len;
+        const int keys_needed = p.full ? (T > 0 ? 1 : 0) : T;  // the causal count needs a key per row
+        const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < keys_needed ||
+                         pt_base < 0 || n_pg < 0 || (int64_t)pt_base + n_pg > p.pt_len;
         if (bad) {
             if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
             return;
@@ -183,7 +184,8 @@ __global__ void __launch_bounds__(kPTThreads, 1)
             p.part_m[at] = -INFINITY;
             p.part_l[at] = 0.f;
             p.part_flag[at] = 0;
-            for (int d = 0; d < D; d += 4) *reinterpret_cast<float4 *>(p.part_o + at * D + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int d = 0; d < D; d += 4)
+                *reinterpret_cast<float4 *>(p.part_o + at * D + d) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         return;
     }
@@ -554,19 +556,22 @@ __global__ void __launch_bounds__(kPTThreads, 1)
                 if (PARTIAL) {
                     float4 *dst = reinterpret_cast<float4 *>(p.part_o + at * D + d0 + cc * 32);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
+                    for (int w = 0; w < 8; ++w)
+                        dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
                 } else if (p.out_bf16) {
                     uint4 *dst =
                         reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d0 + cc * 32);
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        dst[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]), pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
+                        dst[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]),
+                                            pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
                                             pack_bf16x2(o[8 * w + 4], o[8 * w + 5]),
                                             pack_bf16x2(o[8 * w + 6], o[8 * w + 7]));
                 } else {
                     float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d0 + cc * 32);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
+                    for (int w = 0; w < 8; ++w)
+                        dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
                 }
             }
         }
