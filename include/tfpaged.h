@@ -280,10 +280,10 @@ TF_API tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32
  * entry (else TF_DEV_SPLITS and the entry is skipped).
  */
 TF_API tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *ring_k,
-                       const void *ring_v, int64_t ring_slots_total, int32_t n_kv_heads, int32_t head_dim,
-                       const tf_ring_seg *rsegs, int32_t n_segs, const tf_ring_seg *rsegs_host, float scale, int32_t split_slots,
-                       int32_t n_splits_max, void *workspace, size_t workspace_bytes, float *out, uint8_t *flags,
-                       uint32_t *status, tf_stream_t stream);
+                              const void *ring_v, int64_t ring_slots_total, int32_t n_kv_heads, int32_t head_dim,
+                              const tf_ring_seg *rsegs, int32_t n_segs, const tf_ring_seg *rsegs_host, float scale,
+                              int32_t split_slots, int32_t n_splits_max, void *workspace, size_t workspace_bytes,
+                              float *out, uint8_t *flags, uint32_t *status, tf_stream_t stream);
 
 /* Workspace bytes tf_ring_attn needs for these sizes (0 on bad sizes). */
 TF_API size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max);
