@@ -52,6 +52,9 @@ namespace tfp {
 constexpr int kPTSoftmax = 256;
 constexpr int kPTThreads = kPTSoftmax + 64;   // + an MMA warp and a TMA warp
 constexpr int kPTMmaWarp = kPTSoftmax / 32, kPTTmaWarp = kPTMmaWarp + 1;
+// named barriers: 1 the softmax warps, 2-5 a softmax warp pair, kTmemBar the
+// tensor-memory hand-out to the softmax and MMA warps
+constexpr int kTmemBar = 6;
 constexpr int kQM = 128;                      // queries a CTA (the MMA's M)
 constexpr int kBN = 64;                       // keys a tile
 constexpr int kKVSlab = kBN * 128;            // 64 key rows x 128 bytes
@@ -59,14 +62,23 @@ constexpr int kKVStages = 3;                  // K and V buffers in flight
 // tensor-memory columns: two S tiles, Q (D/2 columns of bf16 pairs), O
 constexpr uint32_t kColS0 = 0, kColS1 = 64, kColQ = 128, kColO = 256;
 
-template <int D>
+// Split-KV partials at head dim <= 128 run two CTAs to an SM: both fit in
+// registers and shared memory, and while one holds the tensor memory the other
+// starts (barriers, page ids, its first K/V stages, Q into registers) and
+// waits in the allocation.  A prompt chunk's CTA has the SM to itself.
+template <int D, bool PARTIAL>
+__host__ __device__ constexpr bool pt_paired() { return PARTIAL && D <= 128; }
+
+template <int D, bool PAIRED>
 struct PTCfg {
     static constexpr int kSlabs = D / 64;
     static constexpr int kKVBytes = kSlabs * kKVSlab;
     // kKVStages K buffers, then kKVStages V buffers, then the page ids
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kKVStages * kKVBytes;
-    static constexpr int kPidCap = 4096;  // page ids held in shared memory (16 KB)
+    // page ids held in shared memory (16 KB; 4 KB, 8,192 keys at pages of 8 or
+    // more, for a split when two CTAs share the SM)
+    static constexpr int kPidCap = PAIRED ? 1024 : 4096;
     static constexpr int kOffPid = 2 * kKVStages * kKVBytes;
     static constexpr int kSmemBytes = kOffPid + kPidCap * 4 + 1024;
     static constexpr uint32_t kTmemCols = 512;
@@ -93,10 +105,10 @@ constexpr int kBarO = kBarPr + 2;                   // [2] P V done
 constexpr int kNumBars = kBarO + 2;
 
 template <int D, bool HILO, bool PARTIAL>
-__global__ void __launch_bounds__(kPTThreads, 1)
+__global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     prompt_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const PromptTcParams p) {
-    using C = PTCfg<D>;
+    using C = PTCfg<D, pt_paired<D, PARTIAL>()>;
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bars[kNumBars];
     __shared__ uint32_t s_tmem;
@@ -200,10 +212,6 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         const int id = p.page_table[pt_base + pg_lo + i];
         pids[i] = (id < 0 || id >= p.n_pages) ? -1 : id;
     }
-    if (warp == 0) {
-        tmem_alloc(smem_u32(&s_tmem), C::kTmemCols);
-        tmem_relinquish();
-    }
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i)
             mbar_init(bar(i), (i == kBarQ || i == kBarPr || i == kBarPr + 1) ? kPTSoftmax / 32u : 1u);
@@ -212,10 +220,20 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         s_abort = 0;
         s_vbad[0] = s_vbad[1] = s_vbad[2] = s_vbad[3] = 0;
     }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = s_tmem;
+    // Tensor memory comes later (take_tmem): the TMA warp needs none and
+    // starts on the K/V stages at once, the softmax warps first fetch Q.
+    uint32_t tmem = 0;
+    auto take_tmem = [&]() {
+        if (warp == 0) {
+            tmem_alloc(smem_u32(&s_tmem), C::kTmemCols);  // waits while another CTA of the SM holds it
+            tmem_relinquish();
+        }
+        tc_fence_before();
+        named_bar_sync(kTmemBar, kPTThreads - 32);  // the softmax warps and the MMA warp
+        tc_fence_after();
+        tmem = s_tmem;
+    };
 
     // every lane of a helper warp waits; the answer is the warp's, so all lanes branch alike
     auto wwait = [&](uint32_t b, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(b, phase, abort_flag)); };
@@ -270,6 +288,7 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         }
     } else if (warp == kPTMmaWarp) {
         // ================= MMA warp: lane 0 issues every tcgen05.mma
+        take_tmem();
         const uint32_t idesc_qk = umma_idesc_bf16(kQM, kBN, false, false);
         const uint32_t idesc_pv = umma_idesc_bf16(kQM, D, false, true);
         // S(t) = Q K(t)^T with Q (the A operand) in tensor memory
@@ -351,8 +370,8 @@ __global__ void __launch_bounds__(kPTThreads, 1)
         const float scale_log2 = p.scale_log2;
         float m_ref = -INFINITY, l_run = 0.f;
         uint32_t emax = 0, tail_bad = 0;
-        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t pair_bar = 2 + quad;  // warps quad and quad + 4
+        uint32_t lane_base = 0;
 
         // Q into tensor memory, the A operand of every QK: this thread's half
         // of its row straight from global memory (bf16 pairs are the operand's
@@ -370,6 +389,8 @@ __global__ void __launch_bounds__(kPTThreads, 1)
                 w[v >> 2][4 * (v & 3) + 2] = x.z;
                 w[v >> 2][4 * (v & 3) + 3] = x.w;
             }
+            take_tmem();
+            lane_base = tmem + ((uint32_t)(quad * 32) << 16);
 #pragma unroll
             for (int c = 0; c < kWH / 16; ++c) tmem_st16(lane_base + kColQ + h * kWH + c * 16, w[c]);
             tmem_wait_st();
@@ -649,12 +670,17 @@ static cudaError_t launch_tc_t(const PromptTcParams &p, const void *k, const voi
     // partials are fp32: P goes in as bf16 hi + lo
     auto kern = PARTIAL ? prompt_tc_kernel<D, true, true>
                         : (p.out_bf16 ? prompt_tc_kernel<D, false, false> : prompt_tc_kernel<D, true, false>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PTCfg<D>::kSmemBytes);
+    using C = PTCfg<D, pt_paired<D, PARTIAL>()>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
+    if (pt_paired<D, PARTIAL>()) {  // all of the unified memory as shared memory, so two CTAs fit
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+    }
     const dim3 grid = PARTIAL ? dim3((unsigned)(p.n_qt * p.n_splits_max), (unsigned)p.hkv, (unsigned)n_segs)
                               : dim3((unsigned)((p.n_rows + RT - 1) / RT), (unsigned)p.hkv);
     if (PARTIAL) {
-        kern<<<grid, kPTThreads, PTCfg<D>::kSmemBytes, st>>>(mk, mv, p);
+        kern<<<grid, kPTThreads, C::kSmemBytes, st>>>(mk, mv, p);
         return cudaGetLastError();
     }
     // A prompt chunk may start while the call before it on the stream (this
@@ -665,7 +691,7 @@ static cudaError_t launch_tc_t(const PromptTcParams &p, const void *k, const voi
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
     cfg.blockDim = dim3(kPTThreads);
-    cfg.dynamicSmemBytes = PTCfg<D>::kSmemBytes;
+    cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
