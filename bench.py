@@ -443,7 +443,13 @@ def e2e_decode(b, run, steps, barrier, max_over_ranks, world):
 
 
 def bench_verify(wl, dev, steps, peaks, traffic):
-    b = wl.shared_verify(3)
+    import paged_kv_cache_segment_b200 as tf
+
+    # the split size the library chooses for this batch on this device
+    b0 = wl.shared_verify(3)
+    split, _ = tf.tf_choose_split_keys(b0.segs, n_q_heads=b0.n_q_heads, n_kv_heads=b0.n_kv_heads,
+                                       head_dim=b0.head_dim)
+    b = wl.shared_verify(3, split_keys=split)
     rows = b.n_rows_total
     logits = wl.verify_logits(3, rows)
     run = DecodeRun(b, dev, logits, copies=8)  # 8 x (151 MB of KV + 17 MB of logits)
@@ -455,8 +461,6 @@ def bench_verify(wl, dev, steps, peaks, traffic):
 
     # the same round as one call (tf_verify_round): merge and argmax launch as
     # programmatic dependents, timed at the round's ends
-    import paged_kv_cache_segment_b200 as tf
-
     def round_call(k):
         x = run.sets[k % len(run.sets)]
         tf.tf_verify_round(x["q"], x["kp"], x["vp"], x["pt"], x["segs"], scale=b.scale, split_keys=b.split_keys,
@@ -473,7 +477,8 @@ def bench_verify(wl, dev, steps, peaks, traffic):
     arg_bytes = rows * 128000 * 2
     out = {
         "verify": {"workload": "shared verify: 8 streams x U{1..16} rows, 16/2 heads, D256, P32, contexts "
-                               "U{2048..16384}, 1024-key partials + merge", "rows": rows,
+                               f"U{{2048..16384}}, {split}-key partials (tf_choose_split_keys) + merge", "rows": rows,
+                   "split_keys": split,
                    "kv_gbs": round(kv / (pms + mms) / 1e6, 2), "ms_per_step": round((pms + mms), 5),
                    "tflops": round(flops / (pms * 1e-3) / 1e12, 2),
                    "roofline": dict(roofline("hbm", kv / (pms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",

@@ -192,6 +192,47 @@ TF_API tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_
                                  uint32_t *status, tf_stream_t stream);
 
 /*
+ * A split size for tf_paged_attn_decode, tf_paged_attn_block and
+ * tf_verify_round on batches of more than 8 queries a kv-head at head dim
+ * 256, which the tcgen05 partial kernel serves with one CTA an SM (one CTA
+ * per stream, kv-head, split and 128-query tile).  Host only: reads the
+ * table, launches nothing.  Source:
+ * #1394 ("lfm2: a cheaper DSpark hold", commit list: a hold's attention
+ * partials take all of its query rows in one wave).
+ *
+ * For each candidate size S (256 to 4,096 keys by 128, then by 1,024 to
+ * 16,384, then doubling, up to the first S that holds the longest stream in
+ * one split) the call lists the kernel's CTAs in launch order, gives each a
+ * cost of its 64-key tiles plus a fixed start-up and epilogue cost of eight
+ * tiles (a CTA with no keys costs nothing), hands them in that order to
+ * whichever of n_sms SMs frees first, and keeps the S whose last SM finishes
+ * first (the larger S on a tie).  Grids of more than 2^22 CTAs are skipped.
+ * The costs model the kernel on a B200 (on a verify batch of 8 streams x
+ * 1-16 rows and 2,048-16,384 keys it chose 1,280 keys, the fastest of the
+ * sizes measured from 1,024 to 1,536, and one wave: 61 us against 78 us at
+ * 1,024); the result is a performance choice only: every split gives the
+ * same attention up to rounding.  Head dims 64 and 128 run two CTAs an SM,
+ * whose overlap this schedule does not describe (on a drafter-block batch it
+ * chose 2,432 keys, 13 % slower than 512), so they are refused.
+ *
+ *  segs_host     host segment table, n_segs entries (n_rows and n_keys are
+ *                read; streams with no rows are ignored)
+ *  n_q_heads, n_kv_heads, head_dim  as for tf_paged_attn_decode
+ *  n_sms         the device's SM count (148 on a B200)
+ *  split_keys    out: the chosen S, a multiple of 128 (256 for a batch with
+ *                no rows or keys)
+ *  n_splits_max  out: ceil(n_keys / S) of the longest stream with rows, >= 1
+ *
+ * Returns TF_ERR_ARG for a null pointer, n_segs < 0, n_sms <= 0, heads <= 0
+ * or a segment with negative rows or keys, TF_ERR_UNSUPPORTED when head_dim
+ * is not 256, n_q_heads is not a multiple of n_kv_heads or 128 is not a
+ * multiple of the group.
+ */
+TF_API tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t n_q_heads,
+                                      int32_t n_kv_heads, int32_t head_dim, int32_t n_sms, int32_t *split_keys,
+                                      int32_t *n_splits_max);
+
+/*
  * Append each stream's new rows' keys and values into its pages: the
  * counterpart of tf_wrows_put in #1653 ("spark25 CUDA: the full layers'
  * caches in pages of the core pool", PR body: the rows kernel writes kr/vr

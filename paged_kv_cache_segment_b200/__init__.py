@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     tf_ring_attn,
     tf_ring_attn_noalloc,
     tf_ring_workspace_bytes,
+    tf_choose_split_keys,
     tf_status_str,
     tf_verify_round,
 )

@@ -25,7 +25,8 @@ TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS = 1, 2, 4, 8
 TF_OUT_F32, TF_OUT_BF16 = 0, 1
 
 EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
-           "tf_ring_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_status_str", "tf_abi_version")
+           "tf_ring_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_choose_split_keys", "tf_status_str",
+           "tf_abi_version")
 # bytes of the scratch array tf_ring_attn_noalloc keeps in the library's device image
 TF_RING_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -66,11 +67,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_ring_workspace_bytes.argtypes = [i32, i32, i32, i32]
     lib.tf_ring_workspace_bytes.restype = sz
     lib.tf_argmax_rows.argtypes = [P, i32, i32, i64, P, P, P]
+    lib.tf_choose_split_keys.argtypes = [P, i32, i32, i32, i32, i32, P, P]
     lib.tf_status_str.argtypes = [ctypes.c_int]
     lib.tf_status_str.restype = ctypes.c_char_p
     lib.tf_abi_version.restype = ctypes.c_int32
     for name in ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
-                 "tf_ring_attn_noalloc", "tf_argmax_rows"):
+                 "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_choose_split_keys"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -244,6 +246,21 @@ def tf_paged_attn_prompt(q, k_pool, v_pool, page_table, seg_host, *, scale, out,
         None if flags is None else _dev(flags, "flags", (torch.uint8,)),
         _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
     _check("tf_paged_attn_prompt", rc)
+
+
+def tf_choose_split_keys(segs_host, *, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                         n_sms: int | None = None) -> tuple[int, int]:
+    """(split_keys, n_splits_max) for a head-dim-256 batch the tcgen05
+    partial kernel serves (tf_choose_split_keys).  n_sms defaults to the
+    current device's."""
+    lib = load()
+    sh = as_segs_np(segs_host)
+    if n_sms is None:
+        n_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    split, n_sp = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("tf_choose_split_keys", lib.tf_choose_split_keys(_host_ptr(sh), len(sh), n_q_heads, n_kv_heads, head_dim, n_sms,
+                                                            ctypes.byref(split), ctypes.byref(n_sp)))
+    return int(split.value), int(n_sp.value)
 
 
 def tf_ring_workspace_bytes(n_segs: int, n_q_heads: int, head_dim: int, n_splits_max: int) -> int:

@@ -1,8 +1,11 @@
 // api.cu - the extern "C" entry points declared in include/tfpaged.h: argument
 // checks on the host, then stream-ordered kernel launches.  Nothing here
-// allocates, synchronizes or keeps state between calls.
+// allocates device memory, synchronizes or keeps state between calls.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <functional>
+#include <vector>
 #include <cuda_runtime.h>
 
 #include "tf_internal.h"
@@ -77,6 +80,39 @@ tf_status ring_merge(const float *po, const float *pm, const float *pl, const ui
     mp.out = out;
     mp.flags = flags;
     return cuda_status(launch_merge(mp, head_dim, true, st));
+}
+
+// Cost of one CTA of the tcgen05 partial kernel at head dim 256, in 64-key tiles: its
+// start-up and epilogue (tensor memory, barriers, Q, the first loads' latency,
+// writing o, m, l) count as this many tiles.  Set from a sweep of split sizes
+// on a verify batch (8 streams x 1-16 rows, contexts 2,048-16,384, D 256):
+// values from 3 to 11 all choose the split that measured fastest there.
+constexpr double kSplitCtaOverheadTiles = 8.0;
+
+// Finish time, in tiles, of the partial kernel's grid for split size S: the
+// CTAs (x = split * n_qt + query tile fastest, then kv-head, then stream) go
+// in launch order to whichever SM frees first.  CTAs with no work cost 0.
+double partial_makespan(const tf_seg *sh, int n_segs, int n_kv_heads, int rt, int n_qt, int S, int n_sp_max,
+                        int n_sms, std::vector<double> &heap) {
+    heap.assign((size_t)n_sms, 0.0);  // a min-heap of SM free times
+    auto take = [&](double cost) {
+        std::pop_heap(heap.begin(), heap.end(), std::greater<double>());
+        heap.back() += cost;
+        std::push_heap(heap.begin(), heap.end(), std::greater<double>());
+    };
+    for (int z = 0; z < n_segs; ++z) {
+        const int T = sh[z].n_rows, N = sh[z].n_keys;
+        const int n_sp = T > 0 ? (N + S - 1) / S : 0;
+        for (int y = 0; y < n_kv_heads; ++y)
+            for (int c = 0; c < n_sp_max; ++c)
+                for (int t = 0; t < n_qt; ++t) {
+                    const int qt = n_qt - 1 - t;
+                    if (c >= n_sp || qt * rt >= T) continue;  // exits at once
+                    const int keys = (c + 1 < n_sp ? S : N - c * S);
+                    take(kSplitCtaOverheadTiles + (keys + 63) / 64);
+                }
+    }
+    return *std::max_element(heap.begin(), heap.end());
 }
 
 }  // namespace
@@ -302,6 +338,49 @@ tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_q_heads
     }
     if (n_logit_rows == 0) return TF_OK;
     return tf_argmax_rows(logits, n_logit_rows, n_cols, ld, ids, id_flags, stream);
+}
+
+tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t n_q_heads, int32_t n_kv_heads,
+                               int32_t head_dim, int32_t n_sms, int32_t *split_keys, int32_t *n_splits_max) {
+    if (n_segs < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || n_sms <= 0 || !split_keys || !n_splits_max ||
+        (n_segs > 0 && !segs_host))
+        return TF_ERR_ARG;
+    // the schedule below is that of one CTA an SM (head dim 256); the two
+    // CTAs an SM of head dims 64 and 128 overlap in a way it does not model
+    if (head_dim != 256) return TF_ERR_UNSUPPORTED;
+    if (n_q_heads % n_kv_heads != 0 || 128 % (n_q_heads / n_kv_heads) != 0) return TF_ERR_UNSUPPORTED;
+    const int rt = 128 / (n_q_heads / n_kv_heads);  // rows a 128-query tile
+    int max_rows = 0, max_keys = 0;
+    for (int s = 0; s < n_segs; ++s) {
+        if (segs_host[s].n_rows < 0 || segs_host[s].n_keys < 0) return TF_ERR_ARG;
+        if (segs_host[s].n_rows == 0) continue;
+        max_rows = std::max(max_rows, segs_host[s].n_rows);
+        max_keys = std::max(max_keys, segs_host[s].n_keys);
+    }
+    int best_s = 256;
+    if (max_rows > 0 && max_keys > 0) {
+        const int n_qt = (max_rows + rt - 1) / rt;
+        std::vector<double> heap;
+        double best_t = -1.0;
+        // candidates: 256 .. 4,096 by 128, then by 1,024 to 16,384, then doubling
+        for (int64_t S = 256; S <= (int64_t)1 << 30;) {
+            const int n_sp_max = (int)((max_keys + S - 1) / S);
+            const int64_t ctas = (int64_t)n_segs * n_kv_heads * n_sp_max * n_qt;
+            if (ctas <= ((int64_t)1 << 22)) {  // larger grids are not simulated
+                const double t = partial_makespan(segs_host, n_segs, n_kv_heads, rt, n_qt, (int)S, n_sp_max, n_sms,
+                                                  heap);
+                if (best_t < 0.0 || t <= best_t) {  // the larger split on a tie
+                    best_t = t;
+                    best_s = (int)S;
+                }
+            }
+            if (S >= max_keys) break;  // one split a stream: larger sizes change nothing
+            S = S < 4096 ? S + 128 : (S < 16384 ? S + 1024 : S * 2);
+        }
+    }
+    *split_keys = best_s;
+    *n_splits_max = max_keys > 0 ? (int32_t)((max_keys + best_s - 1) / best_s) : 1;
+    return TF_OK;
 }
 
 tf_status tf_attn_merge(const float *part_o, const float *part_m, const float *part_l, const uint8_t *part_flag,

@@ -67,3 +67,21 @@ def test_round_without_logits_and_refusals():
                            out=torch.empty(1, device=DEV), flags=torch.empty(1, dtype=torch.uint8, device=DEV),
                            status=status_word(), logits=dev(logits), ids=torch.empty(4, dtype=torch.int32, device=DEV),
                            id_flags=torch.empty(4, dtype=torch.uint8, device=DEV), n_cols=2000)
+
+
+def test_round_at_the_chosen_split(orc):
+    """The split tf_choose_split_keys picks for the shared-verify batch on
+    this device (1,280 keys on 148 SMs: 20 tiles, not a power of two); the
+    round still matches the oracle and flags exactly the planted heads."""
+    b0 = wl.shared_verify(3)
+    split, n_sp = tf.tf_choose_split_keys(b0.segs, n_q_heads=16, n_kv_heads=2, head_dim=256)
+    b = wl.shared_verify(3, split_keys=split)
+    assert b.n_splits_max == n_sp
+    logits = wl.verify_logits(3, int(b.segs[:, 1].sum()), n_cols=32000)
+    out, fl, ids, afl, st = _round(b, logits)
+    assert st == 0
+    ref, rf = orc.paged_attn(b.q, b.k_pool, b.v_pool, b.page_table, b.segs, b.scale)
+    compare_attn(out, fl, ref, rf, what=f"round at {split}-key splits")
+    eids, eflags = orc.argmax_rows(logits)
+    np.testing.assert_array_equal(ids, eids)
+    np.testing.assert_array_equal(afl, eflags)
