@@ -575,9 +575,16 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     // a dependent launch (a verify round's argmax) may start; it waits for
     // this grid's completion before it reads anything
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // A (row, head) takes SL adjacent warps of the block, each a 128-column
+    // slice of o (two at D 256, so a warp holds one round of 16 partials in
+    // registers; one below).  Every output element sees the same arithmetic
+    // in the same order whichever warp holds it.
+    constexpr int SL = D > 128 ? D / 128 : 1;
+    constexpr int DW = D / SL;  // columns a warp
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t u = (int64_t)blockIdx.x * 4 + warp;
-    if (u >= p.n_units) return;
+    const int sl = warp % SL, dbase = sl * DW;
+    const int64_t u = (int64_t)blockIdx.x * (4 / SL) + warp / SL;
+    if (u >= p.n_units) return;  // all warps of a unit leave together
     int64_t out_u = u;
     int C = p.n_parts;
     const float qnan = __int_as_float(0x7fc00000);
@@ -592,9 +599,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
                          e.base < 0 || e.base + e.size > p.ring_slots_total ||
                          (e.n_valid + p.split_slots - 1) / p.split_slots > p.n_parts;
         if (bad) {
-            for (int d0 = lane * 4; d0 < D; d0 += 128)
+            for (int d0 = dbase + lane * 4; d0 < dbase + DW; d0 += 128)
                 *reinterpret_cast<float4 *>(p.out + out_u * D + d0) = make_float4(qnan, qnan, qnan, qnan);
-            if (lane == 0) p.flags[out_u] = 1;
+            if (lane == 0 && sl == 0) p.flags[out_u] = 1;
             return;
         }
         C = (e.n_valid + p.split_slots - 1) / p.split_slots;
@@ -608,7 +615,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     // lane c's (m, l, flag) and every lane's slice of each o row.  An empty
     // partial's o is never multiplied in (its weight selects 0), so its
     // unwritten contents cannot leak into the sum.
-    constexpr int NV = (D + 127) / 128;
+    constexpr int NV = (DW + 127) / 128;
     constexpr int CH = 16;
     float4 acc[NV];
 #pragma unroll
@@ -622,9 +629,10 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
         for (int j = 0; j < CH; ++j)
 #pragma unroll
             for (int k = 0; k < NV; ++k) {
-                const int d0 = k * 128 + lane * 4;
-                v[j][k] = (j < n && d0 < D) ? *reinterpret_cast<const float4 *>(po + (int64_t)(c0 + j) * D + d0)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int d0 = dbase + k * 128 + lane * 4;
+                v[j][k] = (j < n && d0 < dbase + DW)
+                              ? *reinterpret_cast<const float4 *>(po + (int64_t)(c0 + j) * D + d0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         float mc = -INFINITY, lc = 0.f;
         if (lane < n) {
@@ -677,8 +685,8 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     bool nf = !isfinite(L) || !any;
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
-        const int d0 = k * 128 + lane * 4;
-        if (d0 < D) {
+        const int d0 = dbase + k * 128 + lane * 4;
+        if (d0 < dbase + DW) {
             acc[k].x /= L;
             acc[k].y /= L;
             acc[k].z /= L;
@@ -686,16 +694,26 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
             nf |= !isfinite(acc[k].x) || !isfinite(acc[k].y) || !isfinite(acc[k].z) || !isfinite(acc[k].w);
         }
     }
-    f |= __any_sync(0xffffffffu, nf) ? 1u : 0u;
+    uint32_t nfw = __any_sync(0xffffffffu, nf) ? 1u : 0u;
+    if constexpr (SL > 1) {
+        // a nonfinite output in any slice flags the whole head: the unit's
+        // warps swap their findings (a barrier of just those warps)
+        __shared__ uint32_t s_nf[4];
+        if (lane == 0) s_nf[warp] = nfw;
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + warp / SL), "r"(32 * SL) : "memory");
+#pragma unroll
+        for (int i = 0; i < SL; ++i) nfw |= s_nf[(warp / SL) * SL + i];
+    }
+    f |= nfw;
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
-        const int d0 = k * 128 + lane * 4;
-        if (d0 < D) {
+        const int d0 = dbase + k * 128 + lane * 4;
+        if (d0 < dbase + DW) {
             const float4 v = f ? make_float4(qnan, qnan, qnan, qnan) : acc[k];
             *reinterpret_cast<float4 *>(p.out + out_u * D + d0) = v;
         }
     }
-    if (lane == 0) p.flags[out_u] = (uint8_t)(f ? 1 : 0);
+    if (lane == 0 && sl == 0) p.flags[out_u] = (uint8_t)(f ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -731,7 +749,8 @@ cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bo
 template <int D, bool RING>
 static cudaError_t launch_merge_t(const MergeParams &p, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)((p.n_units + 3) / 4));
+    constexpr int units = D > 128 ? 4 / (D / 128) : 4;  // (row, head) units a 128-thread block
+    cfg.gridDim = dim3((unsigned)((p.n_units + units - 1) / units));
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
