@@ -206,7 +206,9 @@ TF_API tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_
  * cost of its 64-key tiles plus a fixed start-up and epilogue cost of eight
  * tiles (a CTA with no keys costs nothing), hands them in that order to
  * whichever of n_sms SMs frees first, and keeps the S whose last SM finishes
- * first (the larger S on a tie).  Grids of more than 2^22 CTAs are skipped.
+ * first (the larger S on a tie).  Grids of more than 2^18 CTAs are not
+ * simulated; when no candidate's grid is that small, the call returns the
+ * first S that holds the longest stream in one split (the fewest CTAs).
  * The costs model the kernel on a B200 (on a verify batch of 8 streams x
  * 1-16 rows and 2,048-16,384 keys it chose 1,280 keys, the fastest of the
  * sizes measured from 1,024 to 1,536, and one wave: 61 us against 78 us at

@@ -88,6 +88,9 @@ tf_status ring_merge(const float *po, const float *pm, const float *pl, const ui
 // on a verify batch (8 streams x 1-16 rows, contexts 2,048-16,384, D 256):
 // values from 3 to 11 all choose the split that measured fastest there.
 constexpr double kSplitCtaOverheadTiles = 8.0;
+// Grids larger than this are not simulated (a batch that big fills the SMs
+// many times over whatever the split), which bounds the call's host time.
+constexpr int64_t kSplitMaxSimulatedCtas = (int64_t)1 << 18;
 
 // Finish time, in tiles, of the partial kernel's grid for split size S: the
 // CTAs (x = split * n_qt + query tile fastest, then kv-head, then stream) go
@@ -366,7 +369,7 @@ tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t 
         for (int64_t S = 256; S <= (int64_t)1 << 30;) {
             const int n_sp_max = (int)((max_keys + S - 1) / S);
             const int64_t ctas = (int64_t)n_segs * n_kv_heads * n_sp_max * n_qt;
-            if (ctas <= ((int64_t)1 << 22)) {  // larger grids are not simulated
+            if (ctas <= kSplitMaxSimulatedCtas) {
                 const double t = partial_makespan(segs_host, n_segs, n_kv_heads, rt, n_qt, (int)S, n_sp_max, n_sms,
                                                   heap);
                 if (best_t < 0.0 || t <= best_t) {  // the larger split on a tie
@@ -374,7 +377,10 @@ tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t 
                     best_s = (int)S;
                 }
             }
-            if (S >= max_keys) break;  // one split a stream: larger sizes change nothing
+            if (S >= max_keys) {  // one split a stream: larger sizes change nothing
+                if (best_t < 0.0) best_s = (int)S;  // nothing simulated: the fewest CTAs
+                break;
+            }
             S = S < 4096 ? S + 128 : (S < 16384 ? S + 1024 : S * 2);
         }
     }

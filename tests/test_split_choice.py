@@ -73,6 +73,18 @@ def test_many_sms_take_the_smallest_split():
     assert choose([[0, 1, 20000, 0, 0]], 8, 8, 100000) == (256, 79)
 
 
+def test_batches_too_large_to_simulate_take_one_split_a_stream():
+    """65,535 one-row streams x 8 kv-heads is 524,280 CTAs even at one split a
+    stream, past the 2^18 the call simulates: it returns the first candidate
+    holding the longest stream (1,000 keys -> 1,024) without simulating."""
+    segs = np.zeros((65535, 5), np.int32)
+    segs[:, 0] = np.arange(65535)
+    segs[:, 1] = 1
+    segs[:, 2] = 1000
+    segs[7, 2] = 900
+    assert choose(segs, 8, 8, 148) == (1024, 1)
+
+
 def test_short_and_empty_batches():
     assert choose([[0, 1, 100, 0, 0]], 8, 2, 148) == (256, 1)
     assert choose(np.zeros((0, 5)), 8, 2, 148) == (256, 1)
