@@ -153,13 +153,18 @@ def test_merge_against_oracle_merge(orc, d):
     pl[2, 1, :] = 0
     pm[2, 1, :] = -np.inf  # no partial holds a key: flagged
     po[3, 0, 2, 5] = np.inf  # a nonfinite o: flagged
+    # one in the last columns too: at D 256 the second of a head's two warps
+    # finds it and the whole head (both halves) must come out flagged NaN
+    po[4, 1, 1, d - 3] = -np.inf
     out = torch.empty((rows, hq, d), device="cuda")
     fl = torch.empty((rows, hq), dtype=torch.uint8, device="cuda")
     tf.tf_attn_merge(dev(po), dev(pm), dev(pl), dev(pf), out, fl)
     ref, rf = orc.merge_all(po.astype(np.float64), pm.astype(np.float64), pl.astype(np.float64), pf)
     assert rf.tolist() == (fl.cpu().numpy()).tolist()
-    assert rf[1, 2] and rf[2, 1] and rf[3, 0] and not rf[0, 0]
-    compare_attn(out.cpu().numpy(), fl.cpu().numpy(), ref, rf, max_abs=1e-4, rel_l2=1e-6, what="merge")
+    assert rf[1, 2] and rf[2, 1] and rf[3, 0] and rf[4, 1] and not rf[0, 0]
+    o = out.cpu().numpy()
+    assert np.isnan(o[3, 0]).all() and np.isnan(o[4, 1]).all()
+    compare_attn(o, fl.cpu().numpy(), ref, rf, max_abs=1e-4, rel_l2=1e-6, what="merge")
 
 
 # ----------------------------------------------------------------------------
