@@ -370,14 +370,16 @@ tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t 
             const int n_sp_max = (int)((max_keys + S - 1) / S);
             const int64_t ctas = (int64_t)n_segs * n_kv_heads * n_sp_max * n_qt;
             if (ctas <= kSplitMaxSimulatedCtas) {
-                const double t = partial_makespan(segs_host, n_segs, n_kv_heads, rt, n_qt, (int)S, n_sp_max, n_sms,
+                // SMs past the grid's CTA count stay idle: the heap needs no more
+                const int slots = (int)std::min<int64_t>(n_sms, std::max<int64_t>(ctas, 1));
+                const double t = partial_makespan(segs_host, n_segs, n_kv_heads, rt, n_qt, (int)S, n_sp_max, slots,
                                                   heap);
                 if (best_t < 0.0 || t <= best_t) {  // the larger split on a tie
                     best_t = t;
                     best_s = (int)S;
                 }
             }
-            if (S >= max_keys) {  // one split a stream: larger sizes change nothing
+            if (S >= max_keys || S >= ((int64_t)1 << 30)) {  // one split a stream: larger sizes change nothing
                 if (best_t < 0.0) best_s = (int)S;  // nothing simulated: the fewest CTAs
                 break;
             }

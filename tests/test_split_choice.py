@@ -85,6 +85,13 @@ def test_batches_too_large_to_simulate_take_one_split_a_stream():
     assert choose(segs, 8, 8, 148) == (1024, 1)
 
 
+def test_an_sm_count_past_the_grid_costs_nothing():
+    """More SMs than CTAs: each CTA has its own SM whatever the count, so
+    2^31 - 1 SMs answer like 100,000 (and allocate nothing of that size)."""
+    segs = [[0, 1, 20000, 0, 0], [1, 4, 3000, 0, 0]]
+    assert choose(segs, 8, 8, 2**31 - 1) == choose(segs, 8, 8, 100000)
+
+
 def test_short_and_empty_batches():
     assert choose([[0, 1, 100, 0, 0]], 8, 2, 148) == (256, 1)
     assert choose(np.zeros((0, 5)), 8, 2, 148) == (256, 1)
