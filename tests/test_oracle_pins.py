@@ -522,6 +522,12 @@ CONTROLS = {
                     "int32_t slot = ((e.head + j) % e.size + e.size) % e.size;"),
     "put_rows_reversed": ("const int32_t j = n_keys - n_rows + i;\n            const int64_t page",
                           "const int32_t j = n_keys - 1 - i;\n            const int64_t page"),
+    "causal_count_short": ("const int32_t n_vis = full ? n_keys : n_keys - n_rows + i + 1;",
+                           "const int32_t n_vis = full ? n_keys : n_keys - n_rows + i;"),
+    "full_ignored": ("const int32_t n_vis = full ? n_keys : n_keys - n_rows + i + 1;",
+                     "const int32_t n_vis = n_keys - n_rows + i + 1;"),
+    "partial_causal_short": ("h / group, a, b, n_keys - n_rows + i + 1, scale,",
+                             "h / group, a, b, n_keys - n_rows + i, scale,"),
 }
 
 
@@ -554,6 +560,9 @@ PIN_FOR = {
     "merge_weight_dropped": lambda o: test_merged_partials_equal_unsplit(o, 0),
     "ring_no_lag": lambda o: test_ring_matches_a_writer(o, 10, 13, 6),
     "put_rows_reversed": lambda o: test_put_rows_matches_the_writer(o, [3, 1, 5], [37, 8, 40], 2, 16, 8),
+    "causal_count_short": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
+    "full_ignored": lambda o: test_full_flag_matches_sdpa_without_mask(o),
+    "partial_causal_short": lambda o: test_paged_partials_follow_the_split_rule(o),
 }
 
 
