@@ -528,6 +528,9 @@ CONTROLS = {
                      "const int32_t n_vis = n_keys - n_rows + i + 1;"),
     "partial_causal_short": ("h / group, a, b, n_keys - n_rows + i + 1, scale,",
                              "h / group, a, b, n_keys - n_rows + i, scale,"),
+    "slot_shifted": ("int32_t slot = j % page_size;", "int32_t slot = (j + 1) % page_size;"),
+    "zeros_by_sign": ("if (best < 0 || v > best_v) {",
+                      "if (best < 0 || v > best_v || (v == best_v && signbit(best_v) && !signbit(v))) {"),
 }
 
 
@@ -563,6 +566,8 @@ PIN_FOR = {
     "causal_count_short": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
     "full_ignored": lambda o: test_full_flag_matches_sdpa_without_mask(o),
     "partial_causal_short": lambda o: test_paged_partials_follow_the_split_rule(o),
+    "slot_shifted": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
+    "zeros_by_sign": lambda o: test_argmax_signed_zero_and_all_equal(o),
 }
 
 
