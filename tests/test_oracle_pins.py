@@ -309,6 +309,26 @@ def test_merge_by_hand():
     assert abs(out[0] - 7 / 4) < 1e-15
 
 
+def test_merge_flags_by_hand(orc):
+    """The merged head is flagged (and NaN) when a partial carries a flag,
+    when no partial holds a key, or when a live partial's o is nonfinite; an
+    empty partial (l = 0) is never read, so NaN there changes nothing."""
+    o = np.array([[1.0, -2.0], [2.0, 4.0]])
+    m = np.array([0.0, math.log(3.0)])
+    l = np.array([1.0, 1.0])
+    out, f = orc.merge(o, m, l, np.array([0, 1], np.uint8))  # a flagged partial
+    assert f == 1 and np.isnan(out).all()
+    out, f = orc.merge(o, np.full(2, -np.inf), np.zeros(2), np.zeros(2, np.uint8))  # no key anywhere
+    assert f == 1 and np.isnan(out).all()
+    bad = o.copy()
+    bad[1, 1] = np.inf  # nonfinite o in a live partial
+    out, f = orc.merge(bad, m, l, np.zeros(2, np.uint8))
+    assert f == 1 and np.isnan(out).all()
+    empty = np.array([[1.0, -2.0], [np.nan, np.nan]])  # the second partial holds no key
+    out, f = orc.merge(empty, np.array([0.0, -np.inf]), np.array([1.0, 0.0]), np.zeros(2, np.uint8))
+    assert f == 0 and out.tolist() == [1.0, -2.0]
+
+
 @pytest.mark.parametrize("seed", [0, 1, 2])
 def test_merged_partials_equal_unsplit(orc, seed):
     rng = np.random.default_rng(seed)
@@ -529,6 +549,8 @@ CONTROLS = {
     "partial_causal_short": ("h / group, a, b, n_keys - n_rows + i + 1, scale,",
                              "h / group, a, b, n_keys - n_rows + i, scale,"),
     "slot_shifted": ("int32_t slot = j % page_size;", "int32_t slot = (j + 1) % page_size;"),
+    "merge_flag_dropped": ("        if (flag[c]) bad = 1;\n", "        (void)flag[c];\n"),
+    "merge_reads_empty": ("        if (!(l[c] > 0.0)) continue;\n        double w", "        double w"),
     "zeros_by_sign": ("if (best < 0 || v > best_v) {",
                       "if (best < 0 || v > best_v || (v == best_v && signbit(best_v) && !signbit(v))) {"),
 }
@@ -567,6 +589,8 @@ PIN_FOR = {
     "full_ignored": lambda o: test_full_flag_matches_sdpa_without_mask(o),
     "partial_causal_short": lambda o: test_paged_partials_follow_the_split_rule(o),
     "slot_shifted": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
+    "merge_flag_dropped": lambda o: test_merge_flags_by_hand(o),
+    "merge_reads_empty": lambda o: test_merge_flags_by_hand(o),
     "zeros_by_sign": lambda o: test_argmax_signed_zero_and_all_equal(o),
 }
 
