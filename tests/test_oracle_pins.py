@@ -550,6 +550,10 @@ CONTROLS = {
                              "h / group, a, b, n_keys - n_rows + i, scale,"),
     "slot_shifted": ("int32_t slot = j % page_size;", "int32_t slot = (j + 1) % page_size;"),
     "merge_flag_dropped": ("        if (flag[c]) bad = 1;\n", "        (void)flag[c];\n"),
+    "output_check_dropped": ("        if (!isfinite(out[d])) bad = 1;\n    if (n_vis <= 0) bad = 1;",
+                             "        (void)out[d];\n    if (n_vis <= 0) bad = 1;"),
+    "flagged_output_kept": ("        for (int32_t d = 0; d < head_dim; ++d) out[d] = NAN;\n    *flag = (uint8_t)bad;",
+                            "        (void)out;\n    *flag = (uint8_t)bad;"),
     "merge_reads_empty": ("        if (!(l[c] > 0.0)) continue;\n        double w", "        double w"),
     "zeros_by_sign": ("if (best < 0 || v > best_v) {",
                       "if (best < 0 || v > best_v || (v == best_v && signbit(best_v) && !signbit(v))) {"),
@@ -590,6 +594,8 @@ PIN_FOR = {
     "partial_causal_short": lambda o: test_paged_partials_follow_the_split_rule(o),
     "slot_shifted": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
     "merge_flag_dropped": lambda o: test_merge_flags_by_hand(o),
+    "output_check_dropped": lambda o: test_flags_match_input_level_definition(o),
+    "flagged_output_kept": lambda o: test_flags_match_input_level_definition(o),
     "merge_reads_empty": lambda o: test_merge_flags_by_hand(o),
     "zeros_by_sign": lambda o: test_argmax_signed_zero_and_all_equal(o),
 }
