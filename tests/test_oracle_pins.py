@@ -378,6 +378,12 @@ def test_flags_match_input_level_definition(orc):
     vp[table[b0 + 29 // 8], 1, 29 % 8, 7] = wl.BF16_POS_INF
     b1 = segs[1][3]
     vp[table[b1], 0, 0, 0] = wl.BF16_NAN
+    # K -Inf at stream-1 key 5 head 1 against q[4, 2, 3] = +1: that score is
+    # -Inf, its weight 0 and the output finite, so only the score check can
+    # flag the head (q[4, 3, 3] = -1 makes the other head's score +Inf)
+    kp[table[b1], 1, 5, 3] = wl.BF16_NEG_INF
+    q[4, 2, 3] = 0x3F80  # +1.0
+    q[4, 3, 3] = 0xBF80  # -1.0
     out, flags = orc.paged_attn(q, kp, vp, table, segs, 0.25)
     expect = np.zeros_like(flags)
     for (r0, r, n, base, npg) in segs:
@@ -550,6 +556,7 @@ CONTROLS = {
                              "h / group, a, b, n_keys - n_rows + i, scale,"),
     "slot_shifted": ("int32_t slot = j % page_size;", "int32_t slot = (j + 1) % page_size;"),
     "merge_flag_dropped": ("        if (flag[c]) bad = 1;\n", "        (void)flag[c];\n"),
+    "score_check_dropped": ("        if (!isfinite(s[j])) bad = 1;\n", "        (void)s[j];\n"),
     "output_check_dropped": ("        if (!isfinite(out[d])) bad = 1;\n    if (n_vis <= 0) bad = 1;",
                              "        (void)out[d];\n    if (n_vis <= 0) bad = 1;"),
     "flagged_output_kept": ("        for (int32_t d = 0; d < head_dim; ++d) out[d] = NAN;\n    *flag = (uint8_t)bad;",
@@ -595,6 +602,7 @@ PIN_FOR = {
     "slot_shifted": lambda o: test_paged_attention_matches_sdpa(o, 8, 2, 64, 16),
     "merge_flag_dropped": lambda o: test_merge_flags_by_hand(o),
     "output_check_dropped": lambda o: test_flags_match_input_level_definition(o),
+    "score_check_dropped": lambda o: test_flags_match_input_level_definition(o),
     "flagged_output_kept": lambda o: test_flags_match_input_level_definition(o),
     "merge_reads_empty": lambda o: test_merge_flags_by_hand(o),
     "zeros_by_sign": lambda o: test_argmax_signed_zero_and_all_equal(o),
