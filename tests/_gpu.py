@@ -9,7 +9,7 @@ import paged_kv_cache_segment_b200 as tf
 from paged_kv_cache_segment_b200 import binding
 from paged_kv_cache_segment_b200 import workloads as wl
 
-# spec tolerance for fp32 attention outputs from bf16 inputs
+# the stated tolerance for fp32 attention outputs from bf16 inputs
 MAX_ABS = 2e-3
 REL_L2 = 1e-3
 
