@@ -196,9 +196,9 @@ TF_API tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_
  * tf_verify_round on batches of more than 8 queries a kv-head at head dim
  * 256, which the tcgen05 partial kernel serves with one CTA an SM (one CTA
  * per stream, kv-head, split and 128-query tile).  Host only: reads the
- * table, launches nothing.  Source:
- * #1394 ("lfm2: a cheaper DSpark hold", commit list: a hold's attention
- * partials take all of its query rows in one wave).
+ * table, launches nothing.  Source: #1394 ("lfm2: a cheaper DSpark hold",
+ * commit list: a hold's attention partials take all of its query rows in one
+ * wave).
  *
  * For each candidate size S (256 to 4,096 keys by 128, then by 1,024 to
  * 16,384, then doubling, up to the first S that holds the longest stream in
@@ -225,10 +225,10 @@ TF_API tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_
  *                no rows or keys)
  *  n_splits_max  out: ceil(n_keys / S) of the longest stream with rows, >= 1
  *
- * Returns TF_ERR_ARG for a null pointer, n_segs < 0, n_sms <= 0, heads <= 0
- * or a segment with negative rows or keys, TF_ERR_UNSUPPORTED when head_dim
- * is not 256, n_q_heads is not a multiple of n_kv_heads or 128 is not a
- * multiple of the group.
+ * Returns TF_OK, or TF_ERR_ARG for a null pointer, n_segs < 0, n_sms <= 0,
+ * heads <= 0 or a segment with negative rows or keys, or TF_ERR_UNSUPPORTED
+ * when head_dim is not 256, n_q_heads is not a multiple of n_kv_heads or 128
+ * is not a multiple of the group; the outputs are written only on TF_OK.
  */
 TF_API tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t n_q_heads,
                                       int32_t n_kv_heads, int32_t head_dim, int32_t n_sms, int32_t *split_keys,

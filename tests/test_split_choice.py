@@ -151,6 +151,8 @@ def test_refusals():
     assert call(d=128) == 4  # two CTAs an SM: not the modelled schedule
     assert call(d=64) == 4
     bad = np.array([[0, -1, 100, 0, 0]], np.int32)
+    sp.value, ns.value = -5, -6
     assert call(s=bad.ctypes.data_as(ctypes.c_void_p)) == 1
+    assert (sp.value, ns.value) == (-5, -6)  # outputs are written only on success
     with pytest.raises(binding.TfError):
         choose(segs, 8, 3, 148)
