@@ -22,6 +22,11 @@ RING_SEG_DTYPE = np.dtype(
     [("base", "<i8"), ("q_row", "<i4"), ("size", "<i4"), ("head", "<i4"), ("n_valid", "<i4")]
 )
 
+TREE_SEG_DTYPE = np.dtype(
+    [("base", "<i8"), ("q_row", "<i4"), ("size", "<i4"), ("head", "<i4"), ("n_valid", "<i4"), ("n_nodes", "<i4"),
+     ("parent_base", "<i4")]
+)
+
 ERRORS = {0: "ok", 1: "bad argument", 2: "keys past the stream's pages", 3: "page id outside the pool", 4: "out of memory"}
 
 
@@ -65,6 +70,8 @@ class Oracle:
         L.orc_paged_partials.restype = ctypes.c_int
         L.orc_ring_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, f64, P, P]
         L.orc_ring_attn.restype = ctypes.c_int
+        L.orc_ring_tree_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, f64, P, P]
+        L.orc_ring_tree_attn.restype = ctypes.c_int
         L.orc_argmax_rows.argtypes = [P, i32, i32, i64, P, P]
         L.orc_argmax_rows.restype = None
 
@@ -203,6 +210,25 @@ class Oracle:
         rc = self.lib.orc_ring_attn(self._p(q), rows, hq, self._p(ring_k), self._p(ring_v), slots, hkv, d,
                                     self._p(rs), len(rs), float(scale), self._p(out), self._p(flags))
         self._check(rc, "ring_attn")
+        return out, flags
+
+    def ring_tree_attn(self, q, ring_k, ring_v, tsegs, parents, scale):
+        """Draft trees over rings (orc_ring_tree_attn): float64 out [rows][Hq][D]
+        and uint8 flags [rows][Hq]; rows no tree names stay 0."""
+        q = np.ascontiguousarray(q, np.uint16)
+        ring_k = np.ascontiguousarray(ring_k, np.uint16)
+        ring_v = np.ascontiguousarray(ring_v, np.uint16)
+        ts = np.ascontiguousarray(np.asarray(tsegs).astype(TREE_SEG_DTYPE))
+        par = np.ascontiguousarray(np.asarray(parents, np.int32).reshape(-1))
+        rows, hq, d = q.shape
+        slots, hkv, d2 = ring_k.shape
+        assert d == d2
+        out = np.zeros((rows, hq, d), np.float64)
+        flags = np.zeros((rows, hq), np.uint8)
+        rc = self.lib.orc_ring_tree_attn(self._p(q), rows, hq, self._p(ring_k), self._p(ring_v), slots, hkv, d,
+                                         self._p(ts), len(ts), self._p(par), len(par), float(scale), self._p(out),
+                                         self._p(flags))
+        self._check(rc, "ring_tree_attn")
         return out, flags
 
     # --------------------------------------------------------------- argmax

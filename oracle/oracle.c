@@ -38,6 +38,8 @@
  *  [WR]   #1653, PR body: the rows kernel writes a stream's new K/V rows and
  *         tf_wrows_put copies them into the stream's pages; forward refuses
  *         rows past a slot's pages (PastPages).
+ *  [TREE] #1562, PR body: tf_q36m_attn_tree folds ring slots like the other
+ *         two ring kernels, and a tree equals its chains.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - pool layout [page][kv_head][slot][D], K and V in separate arrays;
@@ -47,7 +49,11 @@
  *    the n before the head, oldest first: slot_j = (head - n + j) mod size;
  *  - a (row, head) is flagged when a score or the output is nonfinite; its
  *    output is then NaN;
- *  - an argmax row holding a NaN or an infinity is flagged and gets id -1.
+ *  - an argmax row holding a NaN or an infinity is flagged and gets id -1;
+ *  - a draft tree's nodes sit in the ring right after its head, node i at
+ *    slot head + i; node i sees the window, then its ancestors from the root
+ *    down, then itself (a chain is then the causal rule over rows written
+ *    after the window).
  */
 #include <math.h>
 #include <stdint.h>
@@ -66,6 +72,16 @@ typedef struct {
     int64_t base;
     int32_t q_row, size, head, n_valid;
 } orc_ring_seg;
+
+/* A tree entry over a ring: the ring is slots [base, base + size); the
+ * window is the n_valid slots before `head`; node i (0 <= i < n_nodes) is
+ * query row q_row + i, its key and value sit at slot (head + i) mod size, and
+ * its parent is parents[parent_base + i] (-1 for a root, else a smaller node
+ * index).  Same field order as the library's struct (32 bytes, no padding). */
+typedef struct {
+    int64_t base;
+    int32_t q_row, size, head, n_valid, n_nodes, parent_base;
+} orc_tree_seg;
 
 /* Exact widening of a bf16 bit pattern. */
 static double bf(uint16_t b)
@@ -460,6 +476,91 @@ int orc_ring_attn(const uint16_t *q, int32_t n_rows_total, int32_t n_q_heads, co
         }
         free(kd);
         free(vd);
+    }
+    return ORC_OK;
+}
+
+/*
+ * Tree attention over a ring ([RING], [TREE]): node i of entry e sees, in this
+ * order, the window slots slot_j = (head - n_valid + j) mod size for
+ * j = 0..n_valid-1 (oldest first), then the nodes on its path from the root
+ * down to itself, node a at slot (head + a) mod size.  The keys of that list
+ * are gathered densely and attended with every q-head of row q_row + i, no
+ * mask.  An entry must have n_nodes >= 1, n_valid >= 0, n_valid + n_nodes <=
+ * size, and -1 <= parent < node for every node; else ORC_ERR_ARG.
+ */
+int orc_ring_tree_attn(const uint16_t *q, int32_t n_rows_total, int32_t n_q_heads, const uint16_t *ring_k,
+                       const uint16_t *ring_v, int64_t slots_total, int32_t n_kv_heads, int32_t head_dim,
+                       const orc_tree_seg *ts, int32_t n_segs, const int32_t *parents, int32_t n_parents,
+                       double scale, double *out, uint8_t *flags)
+{
+    if (n_kv_heads <= 0 || n_q_heads % n_kv_heads != 0) return ORC_ERR_ARG;
+    const int32_t group = n_q_heads / n_kv_heads;
+    for (int32_t s = 0; s < n_segs; ++s) {
+        const orc_tree_seg e = ts[s];
+        if (e.n_nodes < 1 || e.n_valid < 0 || e.size <= 0 || (int64_t)e.n_valid + e.n_nodes > e.size ||
+            e.head < 0 || e.head >= e.size || e.base < 0 || e.base + e.size > slots_total || e.q_row < 0 ||
+            (int64_t)e.q_row + e.n_nodes > n_rows_total || e.parent_base < 0 ||
+            (int64_t)e.parent_base + e.n_nodes > n_parents)
+            return ORC_ERR_ARG;
+        for (int32_t i = 0; i < e.n_nodes; ++i) {
+            const int32_t par = parents[e.parent_base + i];
+            if (par < -1 || par >= i) return ORC_ERR_ARG;
+        }
+    }
+    for (int32_t s = 0; s < n_segs; ++s) {
+        const orc_tree_seg e = ts[s];
+        const int64_t per_key = (int64_t)n_kv_heads * head_dim;
+        const int32_t cap = e.n_valid + e.n_nodes;
+        const int64_t units = (int64_t)e.n_nodes * n_q_heads;
+        int bad_alloc = 0;
+#pragma omp parallel
+        {
+            double *kd = (double *)malloc(sizeof(double) * (size_t)(cap * per_key));
+            double *vd = (double *)malloc(sizeof(double) * (size_t)(cap * per_key));
+            double *qv = (double *)malloc(sizeof(double) * head_dim);
+            double *sc = (double *)malloc(sizeof(double) * (size_t)cap);
+            int32_t *path = (int32_t *)malloc(sizeof(int32_t) * (size_t)e.n_nodes);
+            if (!kd || !vd || !qv || !sc || !path) {
+#pragma omp atomic write
+                bad_alloc = 1;
+            }
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t u = 0; u < units; ++u) {
+                if (bad_alloc) continue;
+                const int32_t i = (int32_t)(u / n_q_heads), h = (int32_t)(u % n_q_heads);
+                /* the node's path, root first */
+                int32_t depth = 0;
+                for (int32_t a = i; a >= 0; a = parents[e.parent_base + a]) path[depth++] = a;
+                int32_t n_keys = 0;
+                for (int32_t j = 0; j < e.n_valid + depth; ++j) {
+                    int32_t slot;
+                    if (j < e.n_valid)
+                        slot = ((e.head - e.n_valid + j) % e.size + e.size) % e.size;
+                    else
+                        slot = (e.head + path[depth - 1 - (j - e.n_valid)]) % e.size;
+                    for (int32_t g = 0; g < n_kv_heads; ++g)
+                        for (int32_t d = 0; d < head_dim; ++d) {
+                            const int64_t src = ((e.base + slot) * n_kv_heads + g) * head_dim + d;
+                            const int64_t dst = ((int64_t)n_keys * n_kv_heads + g) * head_dim + d;
+                            kd[dst] = bf(ring_k[src]);
+                            vd[dst] = bf(ring_v[src]);
+                        }
+                    ++n_keys;
+                }
+                const int64_t row = (int64_t)e.q_row + i;
+                const uint16_t *qs = q + (row * n_q_heads + h) * head_dim;
+                for (int32_t d = 0; d < head_dim; ++d) qv[d] = bf(qs[d]);
+                attend(qv, kd, vd, n_kv_heads, head_dim, h / group, n_keys, scale, sc,
+                       out + (row * n_q_heads + h) * head_dim, flags + row * n_q_heads + h);
+            }
+            free(kd);
+            free(vd);
+            free(qv);
+            free(sc);
+            free(path);
+        }
+        if (bad_alloc) return ORC_ERR_NOMEM;
     }
     return ORC_OK;
 }

@@ -16,6 +16,7 @@ Layouts (all C-contiguous):
 * ``segs``       int32  [S][5] = (q_row, n_rows, n_keys, pt_base, n_pages)
 * ``ring_k``     uint16 (bf16 bits)  [total slots][Hkv][D] (``ring_v`` alike)
 * ``rsegs``      structured array of RING_SEG_DTYPE
+* ``tsegs``      structured array of TREE_SEG_DTYPE, ``parents`` int32
 * ``logits``     uint16 (bf16 bits)  [rows][ld]
 
 The workload shapes follow the pages: many streams' rows in one launch from a
@@ -38,6 +39,14 @@ SEG_FIELDS = ("q_row", "n_rows", "n_keys", "pt_base", "n_pages")
 # Field order chosen so the C struct has no padding: int64 first.
 RING_SEG_DTYPE = np.dtype(
     [("base", "<i8"), ("q_row", "<i4"), ("size", "<i4"), ("head", "<i4"), ("n_valid", "<i4")]
+)
+
+# A draft tree over a ring (32 bytes, no padding): node i of the tree is query
+# row q_row + i, its K/V sit at slot (head + i) mod size, its parent is
+# parents[parent_base + i] (-1 for a root).
+TREE_SEG_DTYPE = np.dtype(
+    [("base", "<i8"), ("q_row", "<i4"), ("size", "<i4"), ("head", "<i4"), ("n_valid", "<i4"), ("n_nodes", "<i4"),
+     ("parent_base", "<i4")]
 )
 
 BF16_NAN = np.uint16(0x7FC0)
@@ -122,6 +131,52 @@ class RingBatch:
 
     def kv_bytes(self) -> int:
         return int(self.rsegs["n_valid"].sum()) * self.n_kv_heads * self.head_dim * 2 * 2
+
+
+@dataclass
+class TreeBatch:
+    """Inputs of one ring tree attention call: every stream's draft tree over
+    its ring (the window is the n_valid slots before the head, the nodes
+    follow the head)."""
+
+    q: np.ndarray
+    ring_k: np.ndarray
+    ring_v: np.ndarray
+    tsegs: np.ndarray
+    parents: np.ndarray
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    scale: float
+    split_slots: int = 512
+    n_splits_max: int = 1
+
+    @property
+    def n_rows_total(self) -> int:
+        return int(self.q.shape[0])
+
+    def kv_bytes(self) -> int:
+        """Algorithmic K+V bytes: the window and every node once per kv-head."""
+        keys = int(self.tsegs["n_valid"].sum() + self.tsegs["n_nodes"].sum())
+        return keys * self.n_kv_heads * self.head_dim * 2 * 2
+
+
+def tree_parents(kind: str, n: int, rng: np.random.Generator) -> list[int]:
+    """Parent indices of an n-node tree in topological order (parent < node,
+    -1 for a root): a chain, several roots (a star), a binary heap, or each
+    node under a uniformly drawn earlier node or the window."""
+    if kind == "chain":
+        return [i - 1 for i in range(n)]
+    if kind == "star":
+        return [-1] * n
+    if kind == "binary":
+        return [(i - 1) // 2 if i > 0 else -1 for i in range(n)]
+    if kind == "random":
+        return [int(rng.integers(-1, i)) for i in range(n)]
+    raise ValueError(kind)
+
+
+TREE_KINDS = ("chain", "star", "binary", "random")
 
 
 def n_splits_for(n_keys: int, split_keys: int, n_splits_max: int, page_size: int) -> int:
@@ -275,6 +330,86 @@ def make_ring_batch(
     )
 
 
+def make_tree_batch(
+    seed: int,
+    n_streams: int,
+    ring_size: int,
+    valid_lo: int,
+    valid_hi: int,
+    nodes_lo: int,
+    nodes_hi: int,
+    n_q_heads: int,
+    n_kv_heads: int,
+    head_dim: int,
+    unused: str = "nan",
+    split_slots: int = 512,
+    kinds: list[str] | None = None,
+    heads: list[int] | None = None,
+    valids: list[int] | None = None,
+    nodes: list[int] | None = None,
+) -> TreeBatch:
+    """``n_streams`` draft trees, each over its own ring of ``ring_size`` slots.
+
+    A ring's write head is drawn at random; its window is the ``n_valid`` slots
+    before the head (U{valid_lo..valid_hi}), and the tree's ``n_nodes``
+    (U{nodes_lo..nodes_hi}) nodes are written at the head and the slots after
+    it, so the window and the nodes wrap whenever they pass the ring's end.
+    Tree shapes cycle through chain, star, binary and random unless ``kinds``
+    is given.  Slots outside the window and the nodes hold ``unused`` data.
+    """
+    rng = np.random.default_rng(seed)
+    if heads is None:
+        heads = [int(h) for h in rng.integers(0, ring_size, size=n_streams)]
+    if nodes is None:
+        nodes = [int(n) for n in rng.integers(nodes_lo, nodes_hi + 1, size=n_streams)]
+    if valids is None:
+        valids = [int(v) for v in rng.integers(valid_lo, valid_hi + 1, size=n_streams)]
+    valids = [min(v, ring_size - n) for v, n in zip(valids, nodes)]
+    if kinds is None:
+        kinds = [TREE_KINDS[s % len(TREE_KINDS)] for s in range(n_streams)]
+    total = n_streams * ring_size
+    shape = (total, n_kv_heads, head_dim)
+    if unused == "normal":
+        ring_k = normal_bf16(rng, shape)
+        ring_v = normal_bf16(rng, shape)
+    else:
+        fill = BF16_NAN if unused == "nan" else np.uint16(0)
+        ring_k = np.full(shape, fill, dtype=np.uint16)
+        ring_v = np.full(shape, fill, dtype=np.uint16)
+    tsegs = np.zeros(n_streams, dtype=TREE_SEG_DTYPE)
+    parents: list[int] = []
+    q_row = 0
+    for s in range(n_streams):
+        base = s * ring_size
+        head, n, t = heads[s], valids[s], nodes[s]
+        tsegs[s] = (base, q_row, ring_size, head, n, t, len(parents))
+        parents += tree_parents(kinds[s], t, rng)
+        q_row += t
+        if unused != "normal":
+            # the window before the head and the nodes from the head on
+            for j in range(-n, t):
+                slot = (head + j) % ring_size
+                ring_k[base + slot] = normal_bf16(rng, (n_kv_heads, head_dim))
+                ring_v[base + slot] = normal_bf16(rng, (n_kv_heads, head_dim))
+    q = normal_bf16(rng, (q_row, n_q_heads, head_dim))
+    keys = [v + t for v, t in zip(valids, nodes)]
+    # a split never crosses the ring's end, so a wrapping range takes one more
+    n_splits_max = max(-(-k // split_slots) + 1 for k in keys)
+    return TreeBatch(
+        q=q,
+        ring_k=ring_k,
+        ring_v=ring_v,
+        tsegs=tsegs,
+        parents=np.asarray(parents, np.int32),
+        n_q_heads=n_q_heads,
+        n_kv_heads=n_kv_heads,
+        head_dim=head_dim,
+        scale=1.0 / math.sqrt(head_dim),
+        split_slots=split_slots,
+        n_splits_max=n_splits_max,
+    )
+
+
 def make_logits(
     seed: int,
     n_rows: int,
@@ -398,6 +533,16 @@ def prompt_chunk_seg(b: PagedBatch, row0: int, row1: int) -> np.ndarray:
     chunk ends at key row1, and its rows are q/out rows row0.. (bookkeeping)."""
     s = b.segs[0]
     return np.array([row0, row1 - row0, row1, s[3], -(-row1 // b.page_size)], dtype=np.int32)
+
+
+def drafter_trees(seed: int = 6, n_streams: int = 17, unused: str = "nan", split_slots: int = 1024) -> TreeBatch:
+    """17 streams, each a draft tree of U{4..16} nodes (chain, star, binary
+    and random shapes in turn) after a window of U{1,000..4,184} slots of its
+    own 4,200-slot ring; 16/2 heads, D 256."""
+    return make_tree_batch(
+        seed, n_streams=n_streams, ring_size=4200, valid_lo=1000, valid_hi=4184, nodes_lo=4, nodes_hi=16,
+        n_q_heads=16, n_kv_heads=2, head_dim=256, unused=unused, split_slots=split_slots,
+    )
 
 
 def drafter_ring(seed: int = 5, n_streams: int = 17, unused: str = "nan", split_slots: int = 256) -> RingBatch:

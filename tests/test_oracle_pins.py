@@ -441,6 +441,146 @@ def test_ring_matches_a_writer(orc, size, written, n_valid):
 
 
 # ----------------------------------------------------------------------------
+# draft trees over a ring
+# ----------------------------------------------------------------------------
+
+def write_tree_ring(rng, size, head, window_k, window_v, node_k, node_v, hkv, d, other=3):
+    """A writer's ring: the window's keys (oldest first) in the slots before
+    `head`, node a in slot head + a (mod size); every other slot NaN; a second
+    ring of `other` slots first, so base != 0."""
+    ring_k = np.full((other + size, hkv, d), wl.BF16_NAN, np.uint16)
+    ring_v = np.full_like(ring_k, wl.BF16_NAN)
+    n = window_k.shape[0]
+    for j in range(n):
+        ring_k[other + (head - n + j) % size] = window_k[j]
+        ring_v[other + (head - n + j) % size] = window_v[j]
+    for a in range(node_k.shape[0]):
+        ring_k[other + (head + a) % size] = node_k[a]
+        ring_v[other + (head + a) % size] = node_v[a]
+    return ring_k, ring_v, other
+
+
+def ancestor_closure(parents):
+    """[T][T] bool: a is node i itself or one of its ancestors, by boolean
+    matrix squaring of (identity | parent edges) until nothing changes."""
+    t = len(parents)
+    m = np.eye(t, dtype=bool)
+    for i, p_ in enumerate(parents):
+        if p_ >= 0:
+            m[i, p_] = True
+    while True:
+        m2 = m | ((m.astype(np.int64) @ m.astype(np.int64)) > 0)
+        if (m2 == m).all():
+            return m
+        m = m2
+
+
+def tree_case(seed, size, head, n_valid, parents, hq=4, hkv=2, d=16):
+    rng = np.random.default_rng(seed)
+    t = len(parents)
+    wk, wv = wl.normal_bf16(rng, (n_valid, hkv, d)), wl.normal_bf16(rng, (n_valid, hkv, d))
+    nk, nv = wl.normal_bf16(rng, (t, hkv, d)), wl.normal_bf16(rng, (t, hkv, d))
+    ring_k, ring_v, base = write_tree_ring(rng, size, head, wk, wv, nk, nv, hkv, d)
+    q = wl.normal_bf16(rng, (t + 2, hq, d))
+    ts = np.zeros(1, oracle.TREE_SEG_DTYPE)
+    ts[0] = (base, 1, size, head, n_valid, t, 2)
+    par = np.array([7, 7] + list(parents), np.int32)  # two unrelated entries first
+    return q, ring_k, ring_v, ts, par, (wk, wv, nk, nv)
+
+
+TREE_SHAPES = [
+    (13, 5, 6, [-1, 0, 1, 2]),                 # a chain, window wraps
+    (16, 0, 9, [-1, -1, -1, -1, -1]),           # a star at head 0: the window wraps from the ring's end
+    (20, 17, 8, [-1, 0, 0, 1, 1, 2, 2]),        # a binary tree whose nodes wrap
+    (12, 4, 0, [-1, 0, -1, 2, 1, 3]),           # no window at all
+    (30, 11, 12, [-1, 0, 1, 0, 3, 3, 5, -1, 7, 2]),
+]
+
+
+@pytest.mark.parametrize("size,head,n_valid,parents", TREE_SHAPES)
+def test_tree_matches_sdpa_with_ancestor_mask(orc, size, head, n_valid, parents):
+    """Node i against float64 SDPA over [window ++ all nodes] with a mask
+    that opens the window and node i's ancestors-or-self (a transitive
+    closure of the parent edges, computed apart from the oracle's walk)."""
+    q, ring_k, ring_v, ts, par, (wk, wv, nk, nv) = tree_case(size * 7 + head, size, head, n_valid, parents)
+    out, flags = orc.ring_tree_attn(q, ring_k, ring_v, ts, par, 0.3)
+    t = len(parents)
+    assert not flags[1:1 + t].any()
+    kf = wl.bf16_bits_to_f32(np.concatenate([wk, nk])).astype(np.float64)
+    vf = wl.bf16_bits_to_f32(np.concatenate([wv, nv])).astype(np.float64)
+    qf = wl.bf16_bits_to_f32(q[1:1 + t]).astype(np.float64)
+    hq, hkv = qf.shape[1], kf.shape[1]
+    mask = np.concatenate([np.ones((t, n_valid), bool), ancestor_closure(parents)], axis=1)
+    qt = torch.from_numpy(qf).permute(1, 0, 2)
+    kt = torch.from_numpy(kf).permute(1, 0, 2).repeat_interleave(hq // hkv, dim=0)
+    vt = torch.from_numpy(vf).permute(1, 0, 2).repeat_interleave(hq // hkv, dim=0)
+    ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.from_numpy(mask), scale=0.3)
+    np.testing.assert_allclose(out[1:1 + t], ref.permute(1, 0, 2).numpy(), rtol=0, atol=TOL)
+    assert not out[0].any() and not out[1 + t:].any()  # rows no tree names are untouched
+
+
+def test_tree_chain_equals_ring_rows(orc):
+    """A tree that is one chain equals, node by node, the ring call whose
+    window runs on through the chain's slots up to that node: the same keys
+    in the same order, so bit for bit."""
+    parents = [-1, 0, 1, 2, 3, 4]
+    q, ring_k, ring_v, ts, par, _ = tree_case(5, 17, 14, 9, parents)
+    out, flags = orc.ring_tree_attn(q, ring_k, ring_v, ts, par, 0.3)
+    e = ts[0]
+    for i in range(len(parents)):
+        rs = np.zeros(1, oracle.RING_SEG_DTYPE)
+        rs[0] = (e["base"], 1 + i, e["size"], (e["head"] + i + 1) % e["size"], e["n_valid"] + i + 1)
+        o2, f2 = orc.ring_attn(q, ring_k, ring_v, rs, 0.3)
+        assert np.array_equal(out[1 + i], o2[1 + i]) and flags[1 + i].tolist() == f2[1 + i].tolist()
+
+
+def test_tree_star_node_equals_window_plus_itself(orc):
+    """A node with no parent sees the window and itself: the ring call over a
+    fresh ring the writer fills with the window and then that node."""
+    parents = [-1, -1, -1, -1]
+    q, ring_k, ring_v, ts, par, (wk, wv, nk, nv) = tree_case(6, 11, 3, 6, parents)
+    out, _ = orc.ring_tree_attn(q, ring_k, ring_v, ts, par, 0.3)
+    rng = np.random.default_rng(0)
+    for i in range(4):
+        rk, rv, base = write_tree_ring(rng, 7, 0, np.concatenate([wk, nk[i:i + 1]]), np.concatenate([wv, nv[i:i + 1]]),
+                                       nk[:0], nv[:0], 2, 16)
+        rs = np.zeros(1, oracle.RING_SEG_DTYPE)
+        rs[0] = (base, 1 + i, 7, 0, 7)
+        o2, _ = orc.ring_attn(q, rk, rv, rs, 0.3)
+        assert np.array_equal(out[1 + i], o2[1 + i])
+
+
+def test_tree_flags_follow_the_paths(orc):
+    """A NaN in node 2's value flags node 2 and the nodes under it, nothing
+    else; an infinity in a window key flags every node."""
+    parents = [-1, 0, 1, 0, 2, 3]  # node 2's subtree: 2, 4
+    q, ring_k, ring_v, ts, par, _ = tree_case(9, 20, 6, 7, parents)
+    e = ts[0]
+    ring_v[e["base"] + (e["head"] + 2) % e["size"], 1, 3] = wl.BF16_NAN
+    _, flags = orc.ring_tree_attn(q, ring_k, ring_v, ts, par, 0.3)
+    want = np.zeros((len(parents), 4), np.uint8)
+    want[[2, 4], 2:4] = 1  # kv-head 1 serves q-heads 2 and 3
+    np.testing.assert_array_equal(flags[1:1 + len(parents)], want)
+    ring_k[e["base"] + (e["head"] - 3) % e["size"], 0, 0] = wl.BF16_POS_INF
+    _, flags = orc.ring_tree_attn(q, ring_k, ring_v, ts, par, 0.3)
+    assert flags[1:1 + len(parents), 0:2].all()
+
+
+def test_tree_refusals(orc):
+    parents = [-1, 0, 1]
+    q, ring_k, ring_v, ts, par, _ = tree_case(3, 10, 2, 4, parents)
+    for bad_par in ([-1, 1, 1], [-1, 0, 3], [0, 0, 1], [-1, -2, 0]):
+        p2 = par.copy()
+        p2[2:] = bad_par
+        with pytest.raises(ValueError):
+            orc.ring_tree_attn(q, ring_k, ring_v, ts, p2, 0.3)
+    ts2 = ts.copy()
+    ts2[0]["n_valid"] = 8  # window + nodes past the ring
+    with pytest.raises(ValueError):
+        orc.ring_tree_attn(q, ring_k, ring_v, ts2, par, 0.3)
+
+
+# ----------------------------------------------------------------------------
 # argmax
 # ----------------------------------------------------------------------------
 
@@ -562,6 +702,15 @@ CONTROLS = {
     "flagged_output_kept": ("        for (int32_t d = 0; d < head_dim; ++d) out[d] = NAN;\n    *flag = (uint8_t)bad;",
                             "        (void)out;\n    *flag = (uint8_t)bad;"),
     "merge_reads_empty": ("        if (!(l[c] > 0.0)) continue;\n        double w", "        double w"),
+    "tree_node_slot_shifted": ("slot = (e.head + path[depth - 1 - (j - e.n_valid)]) % e.size;",
+                               "slot = (e.head + 1 + path[depth - 1 - (j - e.n_valid)]) % e.size;"),
+    "tree_path_without_self": ("for (int32_t a = i; a >= 0; a = parents[e.parent_base + a]) path[depth++] = a;",
+                               "for (int32_t a = parents[e.parent_base + i]; a >= 0; a = parents[e.parent_base + a]) "
+                               "path[depth++] = a;"),
+    "tree_as_chain": ("for (int32_t a = i; a >= 0; a = parents[e.parent_base + a]) path[depth++] = a;",
+                      "for (int32_t a = i; a >= 0; a = a - 1) path[depth++] = a;"),
+    "tree_window_shifted": ("slot = ((e.head - e.n_valid + j) % e.size + e.size) % e.size;\n                    else",
+                            "slot = ((e.head - e.n_valid + 1 + j) % e.size + e.size) % e.size;\n                    else"),
     "zeros_by_sign": ("if (best < 0 || v > best_v) {",
                       "if (best < 0 || v > best_v || (v == best_v && signbit(best_v) && !signbit(v))) {"),
 }
@@ -606,6 +755,10 @@ PIN_FOR = {
     "flagged_output_kept": lambda o: test_flags_match_input_level_definition(o),
     "merge_reads_empty": lambda o: test_merge_flags_by_hand(o),
     "zeros_by_sign": lambda o: test_argmax_signed_zero_and_all_equal(o),
+    "tree_node_slot_shifted": lambda o: test_tree_matches_sdpa_with_ancestor_mask(o, *TREE_SHAPES[2]),
+    "tree_path_without_self": lambda o: test_tree_matches_sdpa_with_ancestor_mask(o, *TREE_SHAPES[4]),
+    "tree_as_chain": lambda o: test_tree_matches_sdpa_with_ancestor_mask(o, *TREE_SHAPES[4]),
+    "tree_window_shifted": lambda o: test_tree_matches_sdpa_with_ancestor_mask(o, *TREE_SHAPES[0]),
 }
 
 
