@@ -344,12 +344,19 @@ TF_API size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t
  * bytes that every GPU which loads the library holds until the process
  * exits.  Arguments and results are tf_ring_attn's, less the workspace.
  *
- *  - Sizes whose tf_ring_workspace_bytes(n_segs, n_q_heads, head_dim,
- *    n_splits_max) exceeds TF_RING_NOALLOC_SCRATCH_BYTES are refused with
- *    TF_ERR_WORKSPACE before anything is launched.
- *  - The first call on a device looks up the scratch array's device address
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture.  Nothing is allocated by this library, then or later.
+ *  - Arguments are checked as tf_ring_attn checks them, with the same
+ *    verdicts; sound arguments whose tf_ring_workspace_bytes(n_segs,
+ *    n_q_heads, head_dim, n_splits_max) exceeds TF_RING_NOALLOC_SCRATCH_BYTES
+ *    are refused with TF_ERR_WORKSPACE.  Nothing is launched on a refusal.
+ *  - Every call looks up the scratch array's address on the current device
+ *    (cudaGetSymbolAddress); TF_ERR_CUDA if that fails.  The library never
+ *    calls cudaMalloc, but the CUDA runtime places the array (and each
+ *    kernel's code) in device memory when it loads this library's device
+ *    code, which under lazy module loading (the CUDA 12 default,
+ *    CUDA_MODULE_LOADING=LAZY) happens on first use.  So make one call on
+ *    each device (n_segs = 0 is enough to place the array; a small real call
+ *    also loads the kernels) before handing the device's memory to a pool,
+ *    and before any stream capture.
  *  - Every call on a device shares the one scratch array and leaves its
  *    partials there.  Nothing in it needs to start at zero (every partial
  *    the merge reads is written first by the same call), but two calls whose
