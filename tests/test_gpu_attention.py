@@ -397,6 +397,30 @@ def test_long_prompt_sampled_rows(orc):
     check_prompt_bf16(r["out"], r["flags"], ref, rf, prompt_bf16_bound(b, ref), sel=sel, what="long prompt")
 
 
+def test_long_prompt_chunk6_and_last_chunk_every_row(orc):
+    """The 15,000-token prompt run as the benchmark runs it (all eight
+    2,048-row chunks back to back, each a programmatic dependent of the one
+    before), then every row and head of chunk 6 (rows 12,288-14,335, the
+    longest full chunk: 12,289-14,336 keys a row, all 64 query tiles of each
+    kv-head) and of the last, ragged chunk (rows 14,336-14,999) against the
+    oracle: the f32 output within max-abs 2e-3 / rel-L2 1e-3, the bf16
+    output within the derived per-element bound and rel-L2 3e-3."""
+    b, spans = wl.long_prompt(4)
+    assert spans[6] == (12288, 14336) and spans[-1] == (14336, 15000)
+    sel = np.zeros((b.n_rows_total, b.n_q_heads), np.uint8)
+    sel[12288:15000, :] = 1
+    ref, rf = orc.paged_attn(b.q, b.k_pool, b.v_pool, b.page_table, b.segs, b.scale, sel=sel)
+    assert not rf[12288:].any()
+    s = sel.astype(bool)
+    r = run_prompt_chunks(b, spans, out_dtype=torch.float32)
+    assert r["status"] == 0
+    compare_attn(r["out"], r["flags"], ref, rf, sel=s, what="long prompt f32, chunk 6 + last")
+    r = run_prompt_chunks(b, spans, out_dtype=torch.bfloat16)
+    assert r["status"] == 0
+    check_prompt_bf16(r["out"], r["flags"], ref, rf, prompt_bf16_bound(b, ref), sel=s,
+                      what="long prompt bf16, chunk 6 + last")
+
+
 @pytest.mark.parametrize("hq,hkv,d,p,n,chunk", [(16, 4, 256, 32, 700, 256), (8, 8, 64, 16, 300, 100),
                                                 (8, 2, 128, 64, 513, 200), (4, 1, 128, 256, 1000, 384),
                                                 (6, 2, 64, 16, 200, 64), (32, 4, 128, 32, 260, 260),
