@@ -38,12 +38,28 @@ def stale() -> bool:
 
 
 def build(verbose_ptxas: bool = False, force: bool = False) -> str:
+    """Compile every csrc/*.cu to an object in parallel (one nvcc a file), then
+    link them into the shared library."""
     if not force and not stale():
         return LIB
-    cmd = [NVCC, *ARCH, *FLAGS, "-I", os.path.join(HERE, "..", "include"), *sources(), "-o", LIB]
-    if verbose_ptxas:
-        cmd += ["-Xptxas", "-v"]
-    subprocess.run(cmd, check=True)
+    from concurrent.futures import ThreadPoolExecutor
+
+    objdir = os.path.join(HERE, "..", "_build")
+    os.makedirs(objdir, exist_ok=True)
+    inc = ["-I", os.path.join(HERE, "..", "include")]
+    compile_flags = [f for f in FLAGS if f != "-shared"]
+
+    def compile_one(src: str) -> str:
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [NVCC, *ARCH, *compile_flags, *inc, "-c", src, "-o", obj]
+        if verbose_ptxas:
+            cmd += ["-Xptxas", "-v"]
+        subprocess.run(cmd, check=True)
+        return obj
+
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, sources()))
+    subprocess.run([NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", LIB], check=True)
     return LIB
 
 
