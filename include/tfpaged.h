@@ -107,6 +107,22 @@ typedef struct {
     int32_t n_valid;
 } tf_ring_seg;
 
+/* One draft tree's entry in a tree table (device array, 32 bytes).  The tree
+ * lives in a ring of slots [base, base + size): its window is the n_valid
+ * slots before `head` (oldest first), node i (0 <= i < n_nodes) is query row
+ * q_row + i and its key and value sit at slot (head + i) mod size, right
+ * after the window; its parent is parents[parent_base + i], -1 for a root
+ * (a child of the window's last slot), else a node index below i. */
+typedef struct {
+    int64_t base;
+    int32_t q_row;
+    int32_t size;
+    int32_t head;
+    int32_t n_valid;
+    int32_t n_nodes;
+    int32_t parent_base;
+} tf_tree_seg;
+
 enum { TF_OUT_F32 = 0, TF_OUT_BF16 = 1 };
 
 /*
@@ -330,6 +346,57 @@ TF_API tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_h
 
 /* Workspace bytes tf_ring_attn needs for these sizes (0 on bad sizes). */
 TF_API size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max);
+
+/*
+ * Draft-tree attention over rings, many trees in one launch: the tree kernel
+ * of #1562 ("Qwen3.6 MTP drafter on CUDA: draft a shared round's streams
+ * together", PR body: tf_q36m_attn_tree folds ring slots in the same groups
+ * and order as the two other ring kernels, and a tree equals its chains).
+ * The page names the kernel only; the layout here is a reading of it.
+ *
+ * Node i of a tree attends, with every q-head of its row, to the tree's
+ * window and then to the nodes on its path from the root down to itself;
+ * no other node.  A tree that is one chain (parent of i = i - 1) gives
+ * node i the ring attention of tf_ring_attn over the n_valid + i + 1 slots
+ * before slot head + i + 1: the causal rule over rows written after the
+ * window.
+ *
+ * The window and the nodes, keys [0, n_valid + n_nodes) from slot
+ * (head - n_valid) mod size on, are split into partials of split_slots keys
+ * that never cross the ring's end: the run before the wrap and the run after
+ * it are cut apart, so a range that wraps takes one partial more than
+ * ceil((n_valid + n_nodes) / split_slots).  The partials merge into out.
+ *
+ *  q          bf16 [n_rows_total][n_q_heads][head_dim]
+ *  ring_k, ring_v  bf16 [ring_slots_total][n_kv_heads][head_dim], 16-byte
+ *             aligned, ring_slots_total <= 2^31 - 65
+ *  tsegs      tf_tree_seg [n_segs] (device); tsegs_host: optional host copy,
+ *             validated (with parents_host, the parents too); the trees' rows
+ *             must not overlap
+ *  parents    int32 [n_parents] (device)
+ *  workspace  device scratch of at least tf_ring_tree_workspace_bytes(...)
+ *             bytes for the partials (by query row); needs no initialisation
+ *  out        f32 [n_rows_total][n_q_heads][head_dim]; flags u8 [rows][Hq]
+ *             (a nonfinite visible score, value or output; the head's out is
+ *             NaN).  Only the trees' rows are written.
+ *
+ * Supported: head_dim in {64, 128, 256}; n_q_heads a multiple of n_kv_heads
+ * whose group G divides 128; 1 <= n_nodes <= 64 a tree; split_slots >= 64.
+ * Device-found errors: a bad entry or a parent outside [-1, node) sets
+ * TF_DEV_BAD_SEG, too few partial slots TF_DEV_SPLITS; the tree's rows are
+ * then flagged NaN.
+ */
+TF_API tf_status tf_ring_tree_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *ring_k,
+                                   const void *ring_v, int64_t ring_slots_total, int32_t n_kv_heads,
+                                   int32_t head_dim, const tf_tree_seg *tsegs, int32_t n_segs,
+                                   const tf_tree_seg *tsegs_host, const int32_t *parents, int32_t n_parents,
+                                   const int32_t *parents_host, float scale, int32_t split_slots,
+                                   int32_t n_splits_max, void *workspace, size_t workspace_bytes, float *out,
+                                   uint8_t *flags, uint32_t *status, tf_stream_t stream);
+
+/* Workspace bytes tf_ring_tree_attn needs (0 on bad sizes). */
+TF_API size_t tf_ring_tree_workspace_bytes(int32_t n_rows_total, int32_t n_q_heads, int32_t head_dim,
+                                           int32_t n_splits_max);
 
 /*
  * tf_ring_attn for callers that cannot allocate device memory.  The pages

@@ -20,6 +20,8 @@ from .binding import (  # noqa: F401
     tf_paged_attn_prompt,
     tf_ring_attn,
     tf_ring_attn_noalloc,
+    tf_ring_tree_attn,
+    tf_ring_tree_workspace_bytes,
     tf_ring_workspace_bytes,
     tf_choose_split_keys,
     tf_status_str,

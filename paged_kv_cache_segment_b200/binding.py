@@ -24,15 +24,20 @@ STATUS_NAMES = {0: "TF_OK", 1: "TF_ERR_ARG", 2: "TF_ERR_PAST_PAGES", 3: "TF_ERR_
 TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS = 1, 2, 4, 8
 TF_OUT_F32, TF_OUT_BF16 = 0, 1
 
-EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
-           "tf_ring_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_choose_split_keys", "tf_status_str",
-           "tf_abi_version")
+EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge",
+           "tf_paged_attn_prompt", "tf_ring_attn", "tf_ring_workspace_bytes", "tf_ring_tree_attn",
+           "tf_ring_tree_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_choose_split_keys",
+           "tf_status_str", "tf_abi_version")
 # bytes of the scratch array tf_ring_attn_noalloc keeps in the library's device image
 TF_RING_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 SEG_DTYPE = np.dtype([("q_row", "<i4"), ("n_rows", "<i4"), ("n_keys", "<i4"), ("pt_base", "<i4"), ("n_pages", "<i4")])
 RING_SEG_DTYPE = np.dtype(
     [("base", "<i8"), ("q_row", "<i4"), ("size", "<i4"), ("head", "<i4"), ("n_valid", "<i4")]
+)
+TREE_SEG_DTYPE = np.dtype(
+    [("base", "<i8"), ("q_row", "<i4"), ("size", "<i4"), ("head", "<i4"), ("n_valid", "<i4"), ("n_nodes", "<i4"),
+     ("parent_base", "<i4")]
 )
 
 
@@ -64,6 +69,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_paged_attn_prompt.argtypes = [P, i32, i32, P, P, i32, i32, i32, i32, P, i32, P, f32, P, i32, P, P, P]
     lib.tf_ring_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, f32, i32, i32, P, sz, P, P, P, P]
     lib.tf_ring_attn_noalloc.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, f32, i32, i32, P, P, P, P]
+    lib.tf_ring_tree_attn.argtypes = [P, i32, i32, P, P, i64, i32, i32, P, i32, P, P, i32, P, f32, i32, i32, P, sz,
+                                      P, P, P, P]
+    lib.tf_ring_tree_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.tf_ring_tree_workspace_bytes.restype = sz
     lib.tf_ring_workspace_bytes.argtypes = [i32, i32, i32, i32]
     lib.tf_ring_workspace_bytes.restype = sz
     lib.tf_argmax_rows.argtypes = [P, i32, i32, i64, P, P, P]
@@ -72,7 +81,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_status_str.restype = ctypes.c_char_p
     lib.tf_abi_version.restype = ctypes.c_int32
     for name in ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
-                 "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_choose_split_keys"):
+                 "tf_ring_attn_noalloc", "tf_ring_tree_attn", "tf_argmax_rows", "tf_choose_split_keys"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -119,6 +128,15 @@ def as_segs_np(segs) -> np.ndarray:
 
 def as_rsegs_np(rsegs) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(rsegs).astype(RING_SEG_DTYPE))
+
+
+def as_tsegs_np(tsegs) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(tsegs).astype(TREE_SEG_DTYPE))
+
+
+def tsegs_to_device(tsegs, device) -> torch.Tensor:
+    """A tree table as a device byte tensor (32 bytes an entry)."""
+    return torch.from_numpy(as_tsegs_np(tsegs).view(np.uint8).copy()).to(device)
 
 
 def rsegs_to_device(rsegs, device) -> torch.Tensor:
@@ -283,6 +301,34 @@ def tf_ring_attn(q, ring_k, ring_v, rsegs, *, scale, split_slots, n_splits_max, 
                           _dev(out, "out", (torch.float32,)), _dev(flags, "flags", (torch.uint8,)),
                           _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
     _check("tf_ring_attn", rc)
+
+
+def tf_ring_tree_workspace_bytes(n_rows_total: int, n_q_heads: int, head_dim: int, n_splits_max: int) -> int:
+    return int(load().tf_ring_tree_workspace_bytes(n_rows_total, n_q_heads, head_dim, n_splits_max))
+
+
+def tf_ring_tree_attn(q, ring_k, ring_v, tsegs, parents, *, scale, split_slots, n_splits_max, workspace, out, flags,
+                      status, tsegs_host=None, parents_host=None, stream=None):
+    """Draft trees over rings, every tree in one launch (tf_ring_tree_attn).
+    tsegs is a device uint8 tensor holding the table (see tsegs_to_device),
+    parents a device int32 tensor."""
+    lib = load()
+    rows, hq, d = q.shape
+    slots, hkv, d2 = ring_k.shape
+    if d2 != d or tuple(ring_v.shape) != tuple(ring_k.shape):
+        raise ValueError("q / ring head dims disagree")
+    n_segs = tsegs.numel() // TREE_SEG_DTYPE.itemsize
+    th = as_tsegs_np(tsegs_host) if tsegs_host is not None else None
+    ph = np.ascontiguousarray(np.asarray(parents_host, np.int32)) if parents_host is not None else None
+    rc = lib.tf_ring_tree_attn(_dev(q, "q", BF16), rows, hq, _dev(ring_k, "ring_k", BF16),
+                               _dev(ring_v, "ring_v", BF16), slots, hkv, d,
+                               _dev(tsegs, "tsegs", (torch.uint8, torch.int8)), n_segs, _host_ptr(th),
+                               _dev(parents, "parents", (torch.int32,)), parents.numel(), _host_ptr(ph),
+                               float(scale), int(split_slots), int(n_splits_max),
+                               _dev(workspace, "workspace", (torch.uint8,)), workspace.numel(),
+                               _dev(out, "out", (torch.float32,)), _dev(flags, "flags", (torch.uint8,)),
+                               _dev(status, "status", (torch.int32, torch.uint32)), _stream(stream))
+    _check("tf_ring_tree_attn", rc)
 
 
 def tf_ring_attn_noalloc(q, ring_k, ring_v, rsegs, *, scale, split_slots, n_splits_max, out, flags, status,

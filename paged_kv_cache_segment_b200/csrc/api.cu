@@ -79,7 +79,7 @@ tf_status ring_merge(const float *po, const float *pm, const float *pl, const ui
     mp.ring_slots_total = ring_slots_total;
     mp.out = out;
     mp.flags = flags;
-    return cuda_status(launch_merge(mp, head_dim, true, st));
+    return cuda_status(launch_merge(mp, head_dim, kMergeRing, st));
 }
 
 // Cost of one CTA of the tcgen05 partial kernel at head dim 256, in 64-key tiles: its
@@ -250,6 +250,26 @@ static tf_status paged_partials(bool full, const void *q, int32_t n_rows_total, 
     return cuda_status(launch_attn_partial(p, head_dim, false, false, grid, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// The row argmax; `early`: the argmax of a verify round, launched right after
+// this library's merge, which may read the logits before the merge finishes
+// (no kernel of the round writes them).
+static tf_status argmax_call(const void *logits, int32_t n_rows, int32_t n_cols, int64_t ld, int32_t *ids,
+                             uint8_t *flags, bool early, tf_stream_t stream) {
+    if (n_rows < 0 || n_cols <= 0 || ld < n_cols) return TF_ERR_ARG;
+    if (n_rows == 0) return TF_OK;
+    if (!logits || !ids || !flags) return TF_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(logits) & 1u) != 0) return TF_ERR_ALIGN;
+    ArgmaxParams p{};
+    p.logits = static_cast<const uint16_t *>(logits);
+    p.n_rows = n_rows;
+    p.n_cols = n_cols;
+    p.ld = ld;
+    p.ids = ids;
+    p.flags = flags;
+    const bool vec = aligned16(logits) && (ld % 8) == 0;
+    return cuda_status(launch_argmax(p, vec, early, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 extern "C" {
 
 tf_status tf_paged_attn_decode(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
@@ -340,7 +360,10 @@ tf_status tf_verify_round(const void *q, int32_t n_rows_total, int32_t n_q_heads
         if (st != TF_OK) return st;
     }
     if (n_logit_rows == 0) return TF_OK;
-    return tf_argmax_rows(logits, n_logit_rows, n_cols, ld, ids, id_flags, stream);
+    // the merge just launched is this library's: the argmax may read the
+    // logits while it drains
+    const bool after_merge = n_segs > 0 && n_rows_total > 0;
+    return argmax_call(logits, n_logit_rows, n_cols, ld, ids, id_flags, after_merge, stream);
 }
 
 tf_status tf_choose_split_keys(const tf_seg *segs_host, int32_t n_segs, int32_t n_q_heads, int32_t n_kv_heads,
@@ -410,7 +433,7 @@ tf_status tf_attn_merge(const float *part_o, const float *part_m, const float *p
     p.n_rows_total = n_rows_total;
     p.out = out;
     p.flags = flags;
-    return cuda_status(launch_merge(p, head_dim, false, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_merge(p, head_dim, kMergeRows, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tf_status tf_paged_attn_prompt(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *k_pool,
@@ -577,21 +600,102 @@ tf_status tf_ring_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, c
                       ring_slots_total, out, flags, st);
 }
 
+size_t tf_ring_tree_workspace_bytes(int32_t n_rows_total, int32_t n_q_heads, int32_t head_dim, int32_t n_splits_max) {
+    if (n_rows_total < 0 || n_q_heads <= 0 || head_dim <= 0 || n_splits_max <= 0) return 0;
+    const size_t parts = (size_t)n_rows_total * n_q_heads * n_splits_max;
+    const size_t o = parts * head_dim * sizeof(float);
+    const size_t ml = 2 * parts * sizeof(float);
+    return ((o + ml + parts + 255) / 256) * 256;
+}
+
+tf_status tf_ring_tree_attn(const void *q, int32_t n_rows_total, int32_t n_q_heads, const void *ring_k,
+                            const void *ring_v, int64_t ring_slots_total, int32_t n_kv_heads, int32_t head_dim,
+                            const tf_tree_seg *tsegs, int32_t n_segs, const tf_tree_seg *tsegs_host,
+                            const int32_t *parents, int32_t n_parents, const int32_t *parents_host, float scale,
+                            int32_t split_slots, int32_t n_splits_max, void *workspace, size_t workspace_bytes,
+                            float *out, uint8_t *flags, uint32_t *status, tf_stream_t stream) {
+    if (n_rows_total < 0 || n_q_heads <= 0 || n_kv_heads <= 0 || ring_slots_total < 0 || n_segs < 0 ||
+        n_parents < 0 || n_splits_max <= 0 || !std::isfinite(scale))
+        return TF_ERR_ARG;
+    if (n_q_heads % n_kv_heads != 0 || !head_dim_ok(head_dim) || split_slots < 64) return TF_ERR_UNSUPPORTED;
+    const int group = n_q_heads / n_kv_heads;
+    if (!tree_tc_supported(head_dim, group)) return TF_ERR_UNSUPPORTED;
+    // a 64-slot box may start at the last slot: its rows stay below 2^31
+    if (n_segs > 65535 || ring_slots_total > 0x7fffffff - 64) return TF_ERR_UNSUPPORTED;
+    if (n_segs == 0 || n_rows_total == 0) return TF_OK;
+    if (!q || !ring_k || !ring_v || !tsegs || !parents || !workspace || !out || !flags || !status) return TF_ERR_ARG;
+    if (!aligned16(q) || !aligned16(ring_k) || !aligned16(ring_v) || !aligned16(out) || !aligned16(workspace))
+        return TF_ERR_ALIGN;
+    if (workspace_bytes < tf_ring_tree_workspace_bytes(n_rows_total, n_q_heads, head_dim, n_splits_max))
+        return TF_ERR_WORKSPACE;
+    int max_nodes = kTreeMaxNodes;
+    if (tsegs_host) {
+        max_nodes = 1;
+        for (int s = 0; s < n_segs; ++s) {
+            const tf_tree_seg e = tsegs_host[s];
+            if (!tree_seg_ok(e, n_rows_total, n_parents, ring_slots_total)) return TF_ERR_ARG;
+            if (tree_splits(e, split_slots).n_sp > n_splits_max) return TF_ERR_ARG;
+            if (parents_host)
+                for (int i = 0; i < e.n_nodes; ++i) {
+                    const int pa = parents_host[e.parent_base + i];
+                    if (pa < -1 || pa >= i) return TF_ERR_ARG;
+                }
+            max_nodes = std::max(max_nodes, (int)e.n_nodes);
+        }
+    }
+    const int rt = 128 / group;  // rows a 128-query tile
+    const int n_qt = (max_nodes + rt - 1) / rt;
+    if ((int64_t)n_qt * n_splits_max > 0x7fffffff) return TF_ERR_UNSUPPORTED;
+    const size_t parts = (size_t)n_rows_total * n_q_heads * n_splits_max;
+    float *po = static_cast<float *>(workspace);
+    float *pm = po + parts * head_dim;
+    float *pl = pm + parts;
+    uint8_t *pf = reinterpret_cast<uint8_t *>(pl + parts);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    PromptTcParams t{};
+    t.q = static_cast<const uint16_t *>(q);
+    t.hq = n_q_heads;
+    t.hkv = n_kv_heads;
+    t.group = group;
+    t.n_rows_total = n_rows_total;
+    t.scale_log2 = scale * 1.4426950408889634f;
+    t.split_keys = split_slots;
+    t.n_splits_max = n_splits_max;
+    t.n_qt = n_qt;
+    t.part_o = po;
+    t.part_m = pm;
+    t.part_l = pl;
+    t.part_flag = pf;
+    t.status = status;
+    t.tsegs = tsegs;
+    t.parents = parents;
+    t.n_parents = n_parents;
+    t.ring_slots_total = ring_slots_total;
+    if (launch_tree_tc(t, head_dim, ring_k, ring_v, n_segs, st) != cudaSuccess) return TF_ERR_CUDA;
+
+    MergeParams mp{};
+    mp.part_o = po;
+    mp.part_m = pm;
+    mp.part_l = pl;
+    mp.part_flag = pf;
+    mp.n_units = (int64_t)n_segs * max_nodes * n_q_heads;
+    mp.n_parts = n_splits_max;
+    mp.hq = n_q_heads;
+    mp.n_rows_total = n_rows_total;
+    mp.split_slots = split_slots;
+    mp.ring_slots_total = ring_slots_total;
+    mp.tsegs = tsegs;
+    mp.tree_nodes = max_nodes;
+    mp.n_parents = n_parents;
+    mp.out = out;
+    mp.flags = flags;
+    return cuda_status(launch_merge(mp, head_dim, kMergeTree, st));
+}
+
 tf_status tf_argmax_rows(const void *logits, int32_t n_rows, int32_t n_cols, int64_t ld, int32_t *ids,
                          uint8_t *flags, tf_stream_t stream) {
-    if (n_rows < 0 || n_cols <= 0 || ld < n_cols) return TF_ERR_ARG;
-    if (n_rows == 0) return TF_OK;
-    if (!logits || !ids || !flags) return TF_ERR_ARG;
-    if ((reinterpret_cast<uintptr_t>(logits) & 1u) != 0) return TF_ERR_ALIGN;
-    ArgmaxParams p{};
-    p.logits = static_cast<const uint16_t *>(logits);
-    p.n_rows = n_rows;
-    p.n_cols = n_cols;
-    p.ld = ld;
-    p.ids = ids;
-    p.flags = flags;
-    const bool vec = aligned16(logits) && (ld % 8) == 0;
-    return cuda_status(launch_argmax(p, vec, reinterpret_cast<cudaStream_t>(stream)));
+    return argmax_call(logits, n_rows, n_cols, ld, ids, flags, false, stream);
 }
 
 const char *tf_status_str(tf_status s) {

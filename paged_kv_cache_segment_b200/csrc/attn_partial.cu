@@ -569,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, (D == 256) ? 1 : 2) attn_partial_ker
 // rows are then read with independent, predicated loads four partials at a
 // time.  The kernel may be launched as a programmatic dependent of the
 // partial kernel: it waits for that grid before reading.
-template <int D, bool RING>
+template <int D, int MODE>
 __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // a dependent launch (a verify round's argmax) may start; it waits for
@@ -585,10 +585,10 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     const int sl = warp % SL, dbase = sl * DW;
     const int64_t u = (int64_t)blockIdx.x * (4 / SL) + warp / SL;
     if (u >= p.n_units) return;  // all warps of a unit leave together
-    int64_t out_u = u;
+    int64_t out_u = u, pu = u;  // the output row's unit, the partials' unit
     int C = p.n_parts;
     const float qnan = __int_as_float(0x7fc00000);
-    if constexpr (RING) {
+    if constexpr (MODE == kMergeRing) {
         // only rows the table names are written; a bad entry (the partial
         // kernel skipped it) gives a flagged NaN row
         const int64_t s = u / p.hq, h = u - s * p.hq;
@@ -605,11 +605,30 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
             return;
         }
         C = (e.n_valid + p.split_slots - 1) / p.split_slots;
+    } else if constexpr (MODE == kMergeTree) {
+        // unit (s * tree_nodes + i) * Hq + h: node i of tree s; its partials
+        // sit at its query row.  Only the trees' rows are written; an entry
+        // the partial kernel skipped gives flagged NaN rows.
+        const int64_t per = (int64_t)p.tree_nodes * p.hq;
+        const int64_t s = u / per, rem = u - s * per;
+        const int i = (int)(rem / p.hq), h = (int)(rem - (int64_t)i * p.hq);
+        const tf_tree_seg e = p.tsegs[s];
+        if (i >= e.n_nodes || e.q_row < 0 || (int64_t)e.q_row + i >= p.n_rows_total) return;
+        out_u = pu = (int64_t)(e.q_row + i) * p.hq + h;
+        const bool ok = tree_seg_ok(e, p.n_rows_total, p.n_parents, p.ring_slots_total) &&
+                        tree_splits(e, p.split_slots).n_sp <= p.n_parts;
+        if (!ok) {
+            for (int d0 = dbase + lane * 4; d0 < dbase + DW; d0 += 128)
+                *reinterpret_cast<float4 *>(p.out + out_u * D + d0) = make_float4(qnan, qnan, qnan, qnan);
+            if (lane == 0 && sl == 0) p.flags[out_u] = 1;
+            return;
+        }
+        C = tree_splits(e, p.split_slots).n_sp;
     }
-    const float *pm = p.part_m + u * p.n_parts;
-    const float *pl = p.part_l + u * p.n_parts;
-    const uint8_t *pf = p.part_flag + u * p.n_parts;
-    const float *po = p.part_o + u * p.n_parts * D;
+    const float *pm = p.part_m + pu * p.n_parts;
+    const float *pl = p.part_l + pu * p.n_parts;
+    const uint8_t *pf = p.part_flag + pu * p.n_parts;
+    const float *po = p.part_o + pu * p.n_parts * D;
 
     // Everything a chunk of up to 16 partials needs is loaded in one round:
     // lane c's (m, l, flag) and every lane's slice of each o row.  An empty
@@ -746,7 +765,7 @@ cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bo
     return launch_partial_d<Src::kPaged, false>(p, head_dim, grid, st);
 }
 
-template <int D, bool RING>
+template <int D, int MODE>
 static cudaError_t launch_merge_t(const MergeParams &p, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     constexpr int units = D > 128 ? 4 / (D / 128) : 4;  // (row, head) units a 128-thread block
@@ -759,16 +778,26 @@ static cudaError_t launch_merge_t(const MergeParams &p, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, merge_kernel<D, RING>, p);
+    return cudaLaunchKernelEx(&cfg, merge_kernel<D, MODE>, p);
 }
 
-cudaError_t launch_merge(const MergeParams &p, int head_dim, bool ring, cudaStream_t st) {
+template <int D>
+static cudaError_t launch_merge_m(const MergeParams &p, int mode, cudaStream_t st) {
+    switch (mode) {
+        case kMergeRows: return launch_merge_t<D, kMergeRows>(p, st);
+        case kMergeRing: return launch_merge_t<D, kMergeRing>(p, st);
+        case kMergeTree: return launch_merge_t<D, kMergeTree>(p, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_merge(const MergeParams &p, int head_dim, int mode, cudaStream_t st) {
     if (p.n_units == 0) return cudaSuccess;
     cudaError_t e;
     switch (head_dim) {
-        case 64: e = ring ? launch_merge_t<64, true>(p, st) : launch_merge_t<64, false>(p, st); break;
-        case 128: e = ring ? launch_merge_t<128, true>(p, st) : launch_merge_t<128, false>(p, st); break;
-        case 256: e = ring ? launch_merge_t<256, true>(p, st) : launch_merge_t<256, false>(p, st); break;
+        case 64: e = launch_merge_m<64>(p, mode, st); break;
+        case 128: e = launch_merge_m<128>(p, mode, st); break;
+        case 256: e = launch_merge_m<256>(p, mode, st); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;

@@ -104,7 +104,7 @@ constexpr int kBarPr = kBarS + 2;                   // [2] P written, V cleaned 
 constexpr int kBarO = kBarPr + 2;                   // [2] P V done
 constexpr int kNumBars = kBarO + 2;
 
-template <int D, bool HILO, bool PARTIAL>
+template <int D, bool HILO, bool PARTIAL, bool TREE = false>
 __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     prompt_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const PromptTcParams p) {
@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     __shared__ float s_xmax[2][2][kQM];     // [tile parity][column half][row]: the halves' tile maxima
     __shared__ float s_xl[2][kQM];          // [column half][row]: final partial sums
     __shared__ uint32_t s_xbad[2][2][kQM];  // [exchange][column half][row]: nonfinite findings
+    __shared__ int s_par[TREE ? kTreeMaxNodes : 1];  // a draft tree's parents
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the merge that follows may launch now; it waits for this grid to finish
@@ -140,30 +141,65 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     // the table), a tile of 128/G rows and, for partials, a split of the keys
     int q_row = p.q_row, T = p.n_rows, N = p.n_keys, pt_base = p.pt_base, n_pg = p.n_pg;
     int qt, split = 0, key_lo = 0, key_hi_split;
+    // a draft tree (entry blockIdx.z of the tree table): the ring row of the
+    // split's first key, the window's length, the tree's parents' base
+    int64_t t_row0 = 0;
+    int t_valid = 0, t_pbase = 0;
     if constexpr (PARTIAL) {
-        const tf_seg sg = p.segs[blockIdx.z];
-        q_row = sg.q_row;
-        T = sg.n_rows;
-        N = sg.n_keys;
-        pt_base = sg.pt_base;
-        n_pg = sg.n_pages;
         split = (int)blockIdx.x / p.n_qt;
         qt = p.n_qt - 1 - (int)blockIdx.x % p.n_qt;  // the most keys first
-        const int keys_needed = p.full ? (T > 0 ? 1 : 0) : T;  // the causal count needs a key per row
-        const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < keys_needed ||
-                         pt_base < 0 || n_pg < 0 || (int64_t)pt_base + n_pg > p.pt_len;
-        if (bad) {
-            if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
-            return;
-        }
-        if ((int64_t)N > ((int64_t)n_pg << p.log2_page)) {
-            if (tid == 0) atomicOr(p.status, TF_DEV_PAST_PAGES);
-            return;
-        }
-        const int n_sp = (N + p.split_keys - 1) / p.split_keys;
-        if (n_sp > p.n_splits_max) {
-            if (tid == 0) atomicOr(p.status, TF_DEV_SPLITS);
-            return;
+        int n_sp;
+        if constexpr (TREE) {
+            const tf_tree_seg e = p.tsegs[blockIdx.z];
+            if (!tree_seg_ok(e, p.n_rows_total, p.n_parents, p.ring_slots_total)) {
+                if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
+                return;
+            }
+            const TreeSplits ts = tree_splits(e, p.split_keys);
+            if (ts.n_sp > p.n_splits_max) {
+                if (tid == 0) atomicOr(p.status, TF_DEV_SPLITS);
+                return;
+            }
+            q_row = e.q_row;
+            T = e.n_nodes;
+            N = ts.n_keys;
+            t_valid = e.n_valid;
+            t_pbase = e.parent_base;
+            n_sp = ts.n_sp;
+            // splits never cross the ring's end: the run before it, then the run after
+            if (split < ts.sa) {
+                key_lo = split * p.split_keys;
+                key_hi_split = min(ts.na, key_lo + p.split_keys);
+            } else {
+                key_lo = ts.na + (split - ts.sa) * p.split_keys;
+                key_hi_split = min(N, key_lo + p.split_keys);
+            }
+            t_row0 = e.base + (key_lo < ts.wrap_at ? ts.start + key_lo : key_lo - ts.wrap_at);
+        } else {
+            const tf_seg sg = p.segs[blockIdx.z];
+            q_row = sg.q_row;
+            T = sg.n_rows;
+            N = sg.n_keys;
+            pt_base = sg.pt_base;
+            n_pg = sg.n_pages;
+            const int keys_needed = p.full ? (T > 0 ? 1 : 0) : T;  // the causal count needs a key per row
+            const bool bad = q_row < 0 || T < 0 || (int64_t)q_row + T > p.n_rows_total || N < keys_needed ||
+                             pt_base < 0 || n_pg < 0 || (int64_t)pt_base + n_pg > p.pt_len;
+            if (bad) {
+                if (tid == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
+                return;
+            }
+            if ((int64_t)N > ((int64_t)n_pg << p.log2_page)) {
+                if (tid == 0) atomicOr(p.status, TF_DEV_PAST_PAGES);
+                return;
+            }
+            n_sp = (N + p.split_keys - 1) / p.split_keys;
+            if (n_sp > p.n_splits_max) {
+                if (tid == 0) atomicOr(p.status, TF_DEV_SPLITS);
+                return;
+            }
+            key_lo = split * p.split_keys;
+            key_hi_split = min(N, key_lo + p.split_keys);
         }
         if (qt * RT >= T) return;
         if (split >= n_sp) {
@@ -176,18 +212,18 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             }
             return;
         }
-        key_lo = split * p.split_keys;
-        key_hi_split = min(N, key_lo + p.split_keys);
     } else {
         qt = (int)gridDim.x - 1 - lin / (int)gridDim.y;  // the most keys first
         key_hi_split = N;
     }
     const int row0 = qt * RT;  // segment-relative first row
     const int rows_here = min(RT, T - row0);
-    // row i of the segment sees keys [0, causal0 + i) (all N with the full flag)
+    // row i of the segment sees keys [0, causal0 + i) (all N with the full
+    // flag); a tree's node sees the window [0, n_valid) and its path's nodes
     const int causal0 = (PARTIAL && p.full) ? N : N - T + 1;
-    const int key_hi_eff = min(key_hi_split, causal0 + row0 + rows_here - 1);  // keys the last valid row sees
-    const int full_hi = min(key_hi_eff, causal0 + row0);                       // keys every row of the tile sees
+    // keys the last valid row sees, and keys every row of the tile sees
+    const int key_hi_eff = TREE ? key_hi_split : min(key_hi_split, causal0 + row0 + rows_here - 1);
+    const int full_hi = TREE ? min(key_hi_eff, t_valid) : min(key_hi_eff, causal0 + row0);
     const int n_tiles = key_hi_eff > key_lo ? (key_hi_eff - key_lo + kBN - 1) / kBN : 0;
     if (PARTIAL && n_tiles == 0) {
         // no row of the tile sees a key of this split: m = -inf, l = 0, o = 0
@@ -207,10 +243,15 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     // read inside the key loop.
     int *pids = reinterpret_cast<int *>(sbase_ptr + C::kOffPid);
     const int pg_lo = key_lo >> p.log2_page;
-    const int n_pid = min((key_hi_eff + P - 1) >> p.log2_page, n_pg) - pg_lo;
-    for (int i = tid; i < n_pid && i < C::kPidCap; i += kPTThreads) {
-        const int id = p.page_table[pt_base + pg_lo + i];
-        pids[i] = (id < 0 || id >= p.n_pages) ? -1 : id;
+    if constexpr (TREE) {
+        // a tree has no pages; its parents go to shared memory instead
+        for (int i = tid; i < T; i += kPTThreads) s_par[i] = p.parents[t_pbase + i];
+    } else {
+        const int n_pid = min((key_hi_eff + P - 1) >> p.log2_page, n_pg) - pg_lo;
+        for (int i = tid; i < n_pid && i < C::kPidCap; i += kPTThreads) {
+            const int id = p.page_table[pt_base + pg_lo + i];
+            pids[i] = (id < 0 || id >= p.n_pages) ? -1 : id;
+        }
     }
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i)
@@ -254,6 +295,16 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             const uint32_t dst0 = is_v ? sV(s) : sK(s);
             const uint32_t full = bar((is_v ? kBarVFull : kBarKFull) + s);
             const CUtensorMap *map = is_v ? &tmV : &tmK;
+            if constexpr (TREE) {
+                // a split's slots are contiguous: one 64-slot box per slab
+                // (rows past the split read neighbouring slots, or zeros past
+                // the arrays, and are masked)
+                if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)C::kKVBytes);
+                __syncwarp();
+                if (lane < C::kSlabs)
+                    tma_load_3d(dst0 + lane * kKVSlab, map, full, 64 * lane, g, (int)(t_row0 + (kt - key_lo)));
+                return;
+            }
             // lane i < n_copies owns box x = i / slabs, slab sl = i % slabs
             const int x = lane / C::kSlabs, sl = lane % C::kSlabs;
             const int key0 = kt + x * BR;
@@ -367,9 +418,37 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
         const int row_i = row0 + qi / G;  // chunk-relative
         const bool valid_row = row_i < T;
         const int lim = valid_row ? min(key_hi_eff, causal0 + row_i) : key_hi_eff;
+        // a tree node's path: bit a set for each node a on it (itself
+        // included), walked up the parents in shared memory; a parent outside
+        // [-1, node) makes the row bad.  Rows past the tree see everything.
+        uint64_t anc = ~0ull;
+        uint32_t path_bad = 0;
+        if constexpr (TREE) {
+            if (valid_row) {
+                anc = 0;
+                for (int a = row_i, steps = 0; a >= 0 && steps < kTreeMaxNodes; ++steps) {
+                    anc |= 1ull << a;
+                    const int pa = s_par[a];
+                    if (pa < -1 || pa >= a) {
+                        path_bad = 1;
+                        break;
+                    }
+                    a = pa;
+                }
+            }
+            if (__any_sync(0xffffffffu, path_bad != 0) && lane == 0) atomicOr(p.status, TF_DEV_BAD_SEG);
+        }
+        // key k is seen by this thread's row: the causal count, or a tree
+        // node's window and path
+        auto visible = [&](int k) -> bool {
+            if constexpr (TREE)
+                return k < key_hi_eff && (k < t_valid || ((anc >> (unsigned)(k - t_valid)) & 1ull) != 0);
+            else
+                return k < lim;
+        };
         const float scale_log2 = p.scale_log2;
         float m_ref = -INFINITY, l_run = 0.f;
-        uint32_t emax = 0, tail_bad = 0;
+        uint32_t emax = 0, tail_bad = path_bad;
         const uint32_t pair_bar = 2 + quad;  // warps quad and quad + 4
         uint32_t lane_base = 0;
 
@@ -421,7 +500,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             if (kt + kBN > full_hi) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const bool vis = kh + c < lim;
+                    const bool vis = visible(kh + c);
                     emax = max(emax, vis ? exp_bits(sv[c]) : 0u);
                     sv[c] = vis ? sv[c] : -INFINITY;
                     m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
@@ -537,7 +616,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
                         }
                     }
                     for (int r = 0; r < kBN; ++r)
-                        if (((((r < 32) ? vb0 : vb1) >> (r & 31)) & 1u) && kt + r < lim) tail_bad = 1;
+                        if (((((r < 32) ? vb0 : vb1) >> (r & 31)) & 1u) && visible(kt + r)) tail_bad = 1;
                 }
                 fence_proxy_async_smem();
             }
@@ -721,6 +800,46 @@ cudaError_t launch_partial_tc(const PromptTcParams &p, int head_dim, const void 
         case 64: return launch_tc_t<64, true>(p, k, v, n_segs, st);
         case 128: return launch_tc_t<128, true>(p, k, v, n_segs, st);
         case 256: return launch_tc_t<256, true>(p, k, v, n_segs, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+bool tree_tc_supported(int head_dim, int group) {
+    return (head_dim == 64 || head_dim == 128 || head_dim == 256) && group >= 1 && group <= 128 &&
+           (128 % group) == 0;
+}
+
+// Draft trees: the partial kernel with ring addressing (a 3-D tensor map over
+// [slots][Hkv][D], boxes of 64 slots) and the ancestor mask on the nodes.
+template <int D>
+static cudaError_t launch_tree_t(const PromptTcParams &p, const void *k, const void *v, int n_segs,
+                                 cudaStream_t st) {
+    CUtensorMap mk, mv;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)p.hkv, (cuuint64_t)p.ring_slots_total};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)p.hkv * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kBN};
+    if (!make_tensor_map_bf16(&mk, k, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&mv, v, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    auto kern = prompt_tc_kernel<D, true, true, true>;
+    using C = PTCfg<D, pt_paired<D, true>()>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (pt_paired<D, true>()) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+    }
+    const dim3 grid((unsigned)(p.n_qt * p.n_splits_max), (unsigned)p.hkv, (unsigned)n_segs);
+    kern<<<grid, kPTThreads, C::kSmemBytes, st>>>(mk, mv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tree_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, int n_segs,
+                           cudaStream_t st) {
+    if (n_segs == 0) return cudaSuccess;
+    switch (head_dim) {
+        case 64: return launch_tree_t<64>(p, k, v, n_segs, st);
+        case 128: return launch_tree_t<128>(p, k, v, n_segs, st);
+        case 256: return launch_tree_t<256>(p, k, v, n_segs, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -44,6 +44,10 @@ struct MergeParams {
     const tf_ring_seg *rsegs;  // ring merge: unit s * Hq + h writes row rsegs[s].q_row
     int split_slots;           // ring merge: partials of entry s are ceil(n_valid / split_slots)
     int64_t ring_slots_total;
+    // tree merge: unit (s * tree_nodes + i) * Hq + h writes row tsegs[s].q_row + i
+    const tf_tree_seg *tsegs;
+    int tree_nodes;
+    int n_parents;
     float *out;
     uint8_t *flags;
 };
@@ -66,6 +70,12 @@ struct PromptTcParams {
     float *part_o, *part_m, *part_l;
     uint8_t *part_flag;
     uint32_t *status;
+    // draft trees over rings: one table entry per tree; partials are laid
+    // out by query row like the paged partials
+    const tf_tree_seg *tsegs;
+    const int32_t *parents;
+    int n_parents;
+    int64_t ring_slots_total;
 };
 
 // Parameters of the KV append (rows into their pages).
@@ -108,8 +118,9 @@ struct ArgmaxParams {
 
 cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bool direct, dim3 grid,
                                 cudaStream_t st);
-cudaError_t launch_merge(const MergeParams &p, int head_dim, bool ring, cudaStream_t st);
-cudaError_t launch_argmax(const ArgmaxParams &p, bool vec, cudaStream_t st);
+enum MergeMode { kMergeRows = 0, kMergeRing = 1, kMergeTree = 2 };
+cudaError_t launch_merge(const MergeParams &p, int head_dim, int mode, cudaStream_t st);
+cudaError_t launch_argmax(const ArgmaxParams &p, bool vec, bool early, cudaStream_t st);
 bool prompt_tc_supported(int head_dim, int group, int page_size);
 bool decode_ws_supported(int head_dim, int n_segs);
 cudaError_t launch_decode_ws(const WsParams &p, int head_dim, bool ring, const void *k, const void *v,
@@ -121,5 +132,39 @@ cudaError_t launch_partial_tc(const PromptTcParams &p, int head_dim, const void 
                               cudaStream_t st);
 
 constexpr int kArgmaxCluster = 2;
+
+// The most nodes a draft tree may have (a node's ancestors are a 64-bit mask).
+constexpr int kTreeMaxNodes = 64;
+
+// Splits of a draft tree's keys: the keys [0, n_valid + n_nodes) run from
+// slot start = (head - n_valid) mod size; those at or past wrap_at = size -
+// start sit at slot key - wrap_at.  Splits never cross the wrap: the first
+// run [0, na) and the second [na, N) are cut into split_slots-key pieces.
+struct TreeSplits {
+    int start, wrap_at, n_keys, na, sa, n_sp;
+};
+__host__ __device__ inline TreeSplits tree_splits(const tf_tree_seg &e, int split_slots) {
+    TreeSplits t;
+    t.start = e.head - e.n_valid;
+    if (t.start < 0) t.start += e.size;
+    t.wrap_at = e.size - t.start;
+    t.n_keys = e.n_valid + e.n_nodes;
+    t.na = t.n_keys < t.wrap_at ? t.n_keys : t.wrap_at;
+    t.sa = (t.na + split_slots - 1) / split_slots;
+    t.n_sp = t.sa + (t.n_keys - t.na + split_slots - 1) / split_slots;
+    return t;
+}
+// An entry the tree kernels can read: sizes and ranges only (the parents are
+// checked as each node's path is walked).
+__host__ __device__ inline bool tree_seg_ok(const tf_tree_seg &e, int n_rows_total, int n_parents,
+                                            int64_t ring_slots_total) {
+    return e.n_nodes >= 1 && e.n_nodes <= kTreeMaxNodes && e.n_valid >= 0 && e.size > 0 &&
+           (int64_t)e.n_valid + e.n_nodes <= e.size && e.head >= 0 && e.head < e.size && e.base >= 0 &&
+           e.base + e.size <= ring_slots_total && e.q_row >= 0 && (int64_t)e.q_row + e.n_nodes <= n_rows_total &&
+           e.parent_base >= 0 && (int64_t)e.parent_base + e.n_nodes <= n_parents;
+}
+bool tree_tc_supported(int head_dim, int group);
+cudaError_t launch_tree_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, int n_segs,
+                           cudaStream_t st);
 
 }  // namespace tfp

@@ -122,3 +122,35 @@ def test_host_checks_of_block_and_append():
     ok = np.array([[0, 2, 5, 0, 1]], np.int32)
     assert append(segs_host=ok.ctypes.data_as(ctypes.c_void_p), pt_host=pt.ctypes.data_as(ctypes.c_void_p),
                   pt_len=1) == 3
+
+
+def call_tree(**kw):
+    lib = tf.load()
+    a = dict(q=FAKE, rows=8, hq=8, k=FAKE, v=FAKE, slots=100, hkv=2, d=64, ts=FAKE, n_segs=1, ts_host=None,
+             par=FAKE, n_par=8, par_host=None, scale=0.125, split=64, nsm=3, ws=FAKE, ws_bytes=1 << 30, out=FAKE,
+             flags=FAKE, st=FAKE, stream=None)
+    a.update(kw)
+    return lib.tf_ring_tree_attn(*a.values())
+
+
+def test_host_checks_of_the_tree_call():
+    ts = np.zeros(1, binding.TREE_SEG_DTYPE)
+    ts[0] = (0, 0, 50, 7, 20, 8, 0)
+    par = np.array([-1, 0, 1, 1, 0, -1, 5, 2], np.int32)
+    host = dict(ts_host=ts.ctypes.data_as(ctypes.c_void_p), par_host=par.ctypes.data_as(ctypes.c_void_p))
+    assert call_tree(d=96) == 4  # head dim
+    assert call_tree(hq=6) == 4  # 6 q-heads over 2 kv-heads: a group of 3 does not divide 128
+    assert call_tree(split=32) == 4  # splits of fewer than 64 slots
+    assert call_tree(nsm=0) == 1
+    assert call_tree(n_segs=0) == 0
+    assert call_tree(q=ctypes.c_void_p(0x10008)) == 6
+    assert call_tree(ws_bytes=1000) == 7  # workspace too small
+    assert tf.tf_ring_tree_workspace_bytes(8, 8, 64, 3) == -(-(8 * 8 * 3 * (64 * 4 + 9)) // 256) * 256
+    # host tables: a parent at or past its node, a window plus nodes past the ring, too few partials
+    for bad_par in ([-1, 1, 1, 1, 0, -1, 5, 2], [-1, 0, 1, 1, 0, -1, 7, 2], [-2, 0, 1, 1, 0, -1, 5, 2]):
+        p2 = np.array(bad_par, np.int32)
+        assert call_tree(ts_host=ts.ctypes.data_as(ctypes.c_void_p), par_host=p2.ctypes.data_as(ctypes.c_void_p)) == 1
+    t2 = ts.copy()
+    t2[0]["n_valid"] = 43
+    assert call_tree(ts_host=t2.ctypes.data_as(ctypes.c_void_p), par_host=host["par_host"]) == 1
+    assert call_tree(nsm=1, **host) == 1  # 28 keys that wrap need 2 partials

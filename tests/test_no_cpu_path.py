@@ -52,6 +52,10 @@ CALLS = {
     "tf_ring_attn": lambda: tf.tf_ring_attn(bf(1, 8, 64), bf(40, 2, 64), bf(40, 2, 64), u8(24), scale=0.125,
                                             split_slots=16, n_splits_max=3, workspace=u8(4096), out=f32(1, 8, 64),
                                             flags=u8(1, 8), status=i32(1)),
+    "tf_ring_tree_attn": lambda: tf.tf_ring_tree_attn(bf(3, 8, 64), bf(40, 2, 64), bf(40, 2, 64), u8(32), i32(3),
+                                                      scale=0.125, split_slots=64, n_splits_max=2,
+                                                      workspace=u8(1 << 16), out=f32(3, 8, 64), flags=u8(3, 8),
+                                                      status=i32(1)),
     "tf_ring_attn_noalloc": lambda: tf.tf_ring_attn_noalloc(bf(1, 8, 64), bf(40, 2, 64), bf(40, 2, 64), u8(24),
                                                             scale=0.125, split_slots=16, n_splits_max=3,
                                                             out=f32(1, 8, 64), flags=u8(1, 8), status=i32(1)),
@@ -65,6 +69,7 @@ def test_host_tensors_are_refused(name):
 
 
 def test_every_compute_call_is_covered():
-    host_only = ("tf_status_str", "tf_abi_version", "tf_ring_workspace_bytes", "tf_choose_split_keys")
+    host_only = ("tf_status_str", "tf_abi_version", "tf_ring_workspace_bytes", "tf_ring_tree_workspace_bytes",
+                 "tf_choose_split_keys")
     compute = {n for n in tf.EXPORTS if n not in host_only}
     assert compute == set(CALLS)
