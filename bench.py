@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--only", default="", help="comma list: decode,verify,ring,prompt,argmax,block,append,e2e,cpu")
+    ap.add_argument("--only", default="", help="comma list: decode,verify,ring,tree,prompt,argmax,block,append,e2e,cpu")
     ap.add_argument("--secondary-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--secondary-cpu-seconds", type=float, default=3.0,
@@ -458,6 +458,8 @@ def run_native(args):
             sec.update(bench_verify(wl, dev, ks, peaks, traffic, cs))
         if want(args, "ring"):
             sec["ring"] = bench_ring(wl, tf, dev, ks, peaks, traffic, cs)
+        if want(args, "tree"):
+            sec["tree"] = bench_tree(wl, tf, dev, ks, peaks, traffic, cs)
         if want(args, "prompt"):
             sec["prompt"] = bench_prompt(wl, tf, dev, max(3, ks // 4), peaks, traffic, cs)
         if want(args, "block"):
@@ -479,14 +481,21 @@ def e2e_decode(b, run, steps, barrier, max_over_ranks, world):
     """The decode step through the public API with HOST inputs and outputs:
     pinned q / segment table / page table copied in, partials + merge, the
     output and flags copied back, every step inside the timed region.  The KV
-    pool is the cache: it stays resident on the device (rotating copies)."""
+    pool is the cache: it stays resident on the device (rotating copies).
+
+    As a serving engine runs it, the copies overlap the compute: step k's
+    inputs go in on a copy stream while step k-1 computes, and its results
+    come back on another while step k+1 computes; events order each step's
+    copy-in, compute and copy-out, and three staging buffers each way keep
+    the steps in flight apart.  The timed region runs from before the first
+    copy-in to after the last copy-out."""
     import torch
 
     import paged_kv_cache_segment_b200 as tf
 
-    # one staging buffer each way, as a serving engine keeps them: the step's
-    # inputs (q, segment table, page table) go in with one copy, its results
-    # (output, flags) come back with one copy
+    # one staging buffer each way a step, as a serving engine keeps them: the
+    # step's inputs (q, segment table, page table) go in with one copy, its
+    # results (output, flags) come back with one copy
     def align(n):
         return (n + 255) // 256 * 256
 
@@ -500,60 +509,78 @@ def e2e_decode(b, run, steps, barrier, max_over_ranks, world):
     in_h = torch.from_numpy(stage_in).pin_memory()
     ob, fb = run.out.numel() * 4, run.fl.numel()
     n_out = align(ob) + align(fb)
-    out_h = torch.empty(n_out, dtype=torch.uint8).pin_memory()
     dev = run.out.device
+    nbuf = len(run.sets)
+    out_h = [torch.empty(n_out, dtype=torch.uint8).pin_memory() for _ in range(nbuf)]
     staged = []
     for x in run.sets:
         buf = torch.empty(n_in, dtype=torch.uint8, device=dev)
+        res = torch.empty(n_out, dtype=torch.uint8, device=dev)
         staged.append(dict(buf=buf, q=buf[0:qb].view(torch.int16).view(tuple(b.q.shape)),
                            segs=buf[o_in[1]:o_in[1] + sb].view(torch.int32).view(tuple(b.segs.shape)),
-                           pt=buf[o_in[2]:o_in[2] + pb].view(torch.int32), kp=x["kp"], vp=x["vp"]))
-    res = torch.empty(n_out, dtype=torch.uint8, device=dev)
-    out_d = res[0:ob].view(torch.float32).view(tuple(run.out.shape))
-    fl_d = res[align(ob):align(ob) + fb].view(tuple(run.fl.shape))
+                           pt=buf[o_in[2]:o_in[2] + pb].view(torch.int32), kp=x["kp"], vp=x["vp"], res=res,
+                           out=res[0:ob].view(torch.float32).view(tuple(run.out.shape)),
+                           fl=res[align(ob):align(ob) + fb].view(tuple(run.fl.shape))))
     h2d = qb + sb + pb
     d2h = ob + fb
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = [dict(inp=torch.cuda.Event(), done=torch.cuda.Event(), out=torch.cuda.Event()) for _ in range(nbuf)]
+    used = [False] * nbuf
 
     def step(k):
-        x = staged[k % len(staged)]
-        x["buf"].copy_(in_h, non_blocking=True)
+        i = k % nbuf
+        x, e = staged[i], ev[i]
+        with torch.cuda.stream(s_in):
+            if used[i]:
+                s_in.wait_event(e["done"])  # the step before on this buffer has read its inputs
+            x["buf"].copy_(in_h, non_blocking=True)
+            e["inp"].record(s_in)
+        comp.wait_event(e["inp"])
+        if used[i]:
+            comp.wait_event(e["out"])  # its results have been copied out
         tf.tf_paged_attn_decode(x["q"], x["kp"], x["vp"], x["pt"], x["segs"], scale=b.scale,
                                 split_keys=b.split_keys, n_splits_max=b.n_splits_max, part_o=run.po, part_m=run.pm,
-                                part_l=run.pl, part_flag=run.pf, status=run.st, segs_host=b.segs)
-        tf.tf_attn_merge(run.po, run.pm, run.pl, run.pf, out_d, fl_d)
-        out_h.copy_(res, non_blocking=True)
+                                part_l=run.pl, part_flag=run.pf, status=run.st, segs_host=b.segs, stream=comp)
+        tf.tf_attn_merge(run.po, run.pm, run.pl, run.pf, x["out"], x["fl"], stream=comp)
+        e["done"].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(e["done"])
+            out_h[i].copy_(x["res"], non_blocking=True)
+            e["out"].record(s_out)
+        used[i] = True
 
-    for k in range(3):
-        step(k)
+    def run_steps(n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(comp)
+        s_in.wait_event(t0)
+        for k in range(n):
+            step(k)
+        for e in ev:
+            if used[ev.index(e)]:
+                comp.wait_event(e["out"])
+        t1.record(comp)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
+    run_steps(3)
     barrier()
-    # per-call host time of the binding (two calls a step), timed apart
+    # the binding's host time a step (two calls, the copies and the events)
     t0 = time.perf_counter()
     for k in range(steps):
         step(k)
     host_us = (time.perf_counter() - t0) / steps * 1e6
     barrier()
-    _, total = timed_steps([step], steps)
+    total = run_steps(steps)
     barrier()
     total = max_over_ranks(total)
     ms = total / steps
-    # the same step (copies included) captured in a CUDA graph per input copy
-    # and replayed, as a serving engine runs its decode step
-    replay = graph_replayer(step, len(staged))
-    for k in range(3):
-        replay(k)
-    barrier()
-    _, gtotal = timed_steps([replay], steps)
-    barrier()
-    gms = max_over_ranks(gtotal) / steps
-    del replay
     return {"value": round(world * b.kv_bytes() / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms, 5),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "host_us_per_step": round(host_us, 1),
-            "path": "binding tf_paged_attn_decode + tf_attn_merge; one pinned staging buffer in (q, segment and page "
-                    "tables) and one out (output and flags), both copied on the compute stream every step",
-            "graph": {"value": round(world * b.kv_bytes() / (gms * 1e-3) / 1e9, 2), "ms_per_step": round(gms, 5),
-                      "path": "the same step, copies included, captured once per input copy in a CUDA graph and "
-                              "replayed"}}
+            "path": "binding tf_paged_attn_decode + tf_attn_merge issued every step; one pinned staging buffer in "
+                    "(q, segment and page tables) and one out (output and flags) a step, copied on their own streams "
+                    "so step k's copy-in and step k-1's copy-out overlap the compute"}
 
 
 def oracle_cpu(fn, seconds, value_per_rep, unit, sample):
@@ -679,6 +706,50 @@ def bench_ring(wl, tf, dev, steps, peaks, traffic, cpu_s):
             "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                  traffic.get("decode_ws:drafter_ring")), "cpu_baseline": cpu,
             "launches": 2 * steps, "l2": "3 rotating copies"}
+
+
+def bench_tree(wl, tf, dev, steps, peaks, traffic, cpu_s):
+    """Draft trees over rings: 17 trees of 4-16 nodes (chain, star, binary,
+    random) after windows of 1,000-4,184 slots of their own 4,200-slot rings,
+    16/2 heads, D 256; 3 rotating copies of the rings."""
+    import torch
+
+    import oracle
+    from paged_kv_cache_segment_b200 import binding
+
+    b = wl.drafter_trees(6)
+    rows, hq, d = b.q.shape
+    sets = [dict(q=to_dev(b.q, dev), rk=to_dev(b.ring_k, dev), rv=to_dev(b.ring_v, dev),
+                 ts=binding.tsegs_to_device(b.tsegs, dev), par=to_dev(b.parents, dev)) for _ in range(3)]
+    ws = torch.empty(tf.tf_ring_tree_workspace_bytes(rows, hq, d, b.n_splits_max), dtype=torch.uint8, device=dev)
+    out = torch.empty((rows, hq, d), device=dev)
+    fl = torch.empty((rows, hq), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(k):
+        x = sets[k % 3]
+        tf.tf_ring_tree_attn(x["q"], x["rk"], x["rv"], x["ts"], x["par"], scale=b.scale, split_slots=b.split_slots,
+                             n_splits_max=b.n_splits_max, workspace=ws, out=out, flags=fl, status=st,
+                             tsegs_host=b.tsegs, parents_host=b.parents)
+
+    g = graph_replayer(step, 3)
+    for k in range(3):
+        g(k)
+    _, total = timed_steps([g], steps)
+    ms = total / steps
+    kv = b.kv_bytes()
+    assert int(st.item()) == 0
+    orc = oracle.get()
+    cpu = oracle_cpu(lambda: orc.ring_tree_attn(b.q, b.ring_k, b.ring_v, b.tsegs, b.parents, b.scale), cpu_s,
+                     kv / 1e9, "GB/s", "whole passes of the 17 trees")
+    return {"workload": "drafter trees: 17 trees of U{4..16} nodes (chain/star/binary/random) after windows of "
+                        "U{1000..4184} slots of 4,200-slot rings, 16/2 heads, D256, "
+                        f"{b.split_slots}-slot partials + merge", "nodes": rows,
+            "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2), "ms_per_step": round(ms, 5),
+            "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                                      traffic.get("prompt_tc:drafter_trees")),
+                             kernel="prompt_tc_kernel<256, hilo, partial, tree> + merge (the whole step)"),
+            "cpu_baseline": cpu, "launches": 2 * steps, "l2": "3 rotating copies"}
 
 
 def bench_prompt(wl, tf, dev, steps, peaks, traffic, cpu_s):
