@@ -351,7 +351,8 @@ TF_API size_t tf_ring_workspace_bytes(int32_t n_segs, int32_t n_q_heads, int32_t
  * Draft-tree attention over rings, many trees in one launch: the tree kernel
  * of #1562 ("Qwen3.6 MTP drafter on CUDA: draft a shared round's streams
  * together", PR body: tf_q36m_attn_tree folds ring slots in the same groups
- * and order as the two other ring kernels, and a tree equals its chains).
+ * and order as the two other ring kernels, and a tree checked against its
+ * chains gives their results).
  * The page names the kernel only; the layout here is a reading of it.
  *
  * Node i of a tree attends, with every q-head of its row, to the tree's

@@ -39,7 +39,8 @@
  *         tf_wrows_put copies them into the stream's pages; forward refuses
  *         rows past a slot's pages (PastPages).
  *  [TREE] #1562, PR body: tf_q36m_attn_tree folds ring slots like the other
- *         two ring kernels, and a tree equals its chains.
+ *         two ring kernels, and a tree checked against the chains it is
+ *         made of gives their results.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - pool layout [page][kv_head][slot][D], K and V in separate arrays;

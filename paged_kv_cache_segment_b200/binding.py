@@ -105,8 +105,9 @@ BF16 = (torch.bfloat16, torch.int16, torch.uint16)
 
 
 def _stream(stream) -> int:
+    """The raw cudaStream_t: the given stream, or the current one."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        return torch._C._cuda_getCurrentRawStream(torch.cuda.current_device())
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
@@ -118,7 +119,7 @@ def _check(fn: str, rc: int):
 def _host_ptr(a):
     if a is None:
         return None
-    return a.ctypes.data_as(ctypes.c_void_p)
+    return a.ctypes.data
 
 
 def as_segs_np(segs) -> np.ndarray:

@@ -27,6 +27,7 @@
 //    formed in registers with movmatrix (bf16 hi + bf16 lo, about 16 bits).
 //  - At an item's end the four warps' online-softmax states meet in shared
 //    memory (a two-level tree) and one partial per (row, q-head) is written.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -804,10 +805,25 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
 // host side
 // ---------------------------------------------------------------------------
 
-static int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
+// CTAs of a persistent launch on the current device: its SM count times the
+// CTAs of the kernel an SM holds.  Both are facts of the device and the
+// kernel, so each instance looks them up once per device and keeps them.
+template <int D, bool RING>
+static int ws_grid_cap() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> cap[kMaxDevices];  // 0: not looked up yet
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    const int known = cap[dev].load(std::memory_order_relaxed);
+    if (known > 0) return known;
+    int n = 148, per_sm = 1;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_ws_kernel<D, RING>, WsCfg<D>::kThreads,
+                                                      WsCfg<D>::kSmem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    cap[dev].store(n * per_sm, std::memory_order_relaxed);
+    return n * per_sm;
 }
 
 template <int D, bool RING>
@@ -831,12 +847,7 @@ static cudaError_t launch_ws_t(const WsParams &p, const void *k, const void *v, 
     auto kern = decode_ws_kernel<D, RING>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WsCfg<D>::kSmem);
     if (e != cudaSuccess) return e;
-    int per_sm = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WsCfg<D>::kThreads, WsCfg<D>::kSmem) !=
-            cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    int64_t grid = (int64_t)sm_count() * per_sm;
+    int64_t grid = ws_grid_cap<D, RING>();
     if (n_items_bound < grid) grid = n_items_bound < 1 ? 1 : n_items_bound;
     kern<<<(unsigned)grid, WsCfg<D>::kThreads, WsCfg<D>::kSmem, st>>>(mk, mv, p);
     return cudaGetLastError();

@@ -535,7 +535,7 @@ def prompt_chunk_seg(b: PagedBatch, row0: int, row1: int) -> np.ndarray:
     return np.array([row0, row1 - row0, row1, s[3], -(-row1 // b.page_size)], dtype=np.int32)
 
 
-def drafter_trees(seed: int = 6, n_streams: int = 17, unused: str = "nan", split_slots: int = 1024) -> TreeBatch:
+def drafter_trees(seed: int = 6, n_streams: int = 17, unused: str = "nan", split_slots: int = 768) -> TreeBatch:
     """17 streams, each a draft tree of U{4..16} nodes (chain, star, binary
     and random shapes in turn) after a window of U{1,000..4,184} slots of its
     own 4,200-slot ring; 16/2 heads, D 256."""
