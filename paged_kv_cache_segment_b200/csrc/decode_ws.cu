@@ -269,6 +269,12 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
     }
+    if (!RING && warp == 1) {
+        // the page table's first 16 KB into L2 while warp 0 works out the
+        // items, so the producer's first page-id reads do not go to DRAM
+        const int n = min(p.pt_len, 4096);
+        for (int i = lane * 32; i < n; i += 32 * 32) prefetch_l2(p.page_table + i);
+    }
     if (warp == 0) {
         // per stream: its items (splits x Hkv), its full-length ones, and the
         // tile count of its last split, bucketed for the tail order
@@ -308,13 +314,23 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             prefix_full[p.n_segs] = running_full;
             s_total = running;
             s_full = running_full;
-            // bucket starts in the tail order, longest tails first
-            int at = 0;
-            for (int k = kBuckets - 1; k >= 0; --k) {
-                const int n = s_bucket[k];
-                s_bucket[k] = at;
-                at += n;
+        }
+        {
+            // bucket starts in the tail order, longest tails first: lane l
+            // holds buckets 63 - 2l and 62 - 2l, and an exclusive scan over
+            // the lanes gives each bucket the count of the longer ones
+            const int hi = kBuckets - 1 - 2 * lane, lo = hi - 1;
+            const int n_hi = s_bucket[hi], n_lo = s_bucket[lo];
+            int incl = n_hi + n_lo;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
             }
+            const int before = incl - n_hi - n_lo;
+            __syncwarp();
+            s_bucket[hi] = before;
+            s_bucket[lo] = before + n_hi;
         }
         __syncwarp();
         // each stream with splits takes the next place of its bucket, streams
@@ -382,6 +398,26 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             };
             uint32_t tc = 0, qc = 0;
             bool ok = true;
+            // an item goes to the consumers with its queries (a bulk copy into
+            // the next of the kNQ query buffers); item k + 1 is published as
+            // soon as item k's first tile has gone out, so its queries land
+            // while item k's tiles stream
+            auto publish = [&](const WsItem &w) -> bool {
+                const uint32_t qs = qc % C::kNQ;
+                if (qc >= (uint32_t)C::kNQ && !mbar_wait(smem_u32(&qempty_bar[qs]), ((qc / C::kNQ) - 1) & 1))
+                    return false;
+                if (lane == 0) {
+                    s_item[qs] = w;  // published with the queries (the arrive below releases it)
+                    const uint32_t qdst = sbase + C::kOffQ + qs * C::kQBytes;
+                    const uint32_t qbytes = (uint32_t)(p.group * D * 2);
+                    mbar_arrive_expect_tx(smem_u32(&qfull_bar[qs]), qbytes * w.n_rows);
+                    for (int i = 0; i < w.n_rows; ++i)
+                        bulk_load(qdst + i * qbytes, p.q + ((int64_t)(w.q_row + i) * p.hq + w.g * p.group) * D,
+                                  qbytes, smem_u32(&qfull_bar[qs]));
+                }
+                ++qc;
+                return true;
+            };
             int k = 0, L = ws_snake(0, bid, grid);
             WsItem it{};
             int win = 0, w0 = 0;
@@ -389,6 +425,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                 it = ws_resolve<RING>(p, prefix, prefix_full, tail_order, n_full, L);
                 w0 = it.key_lo >> p.log2_page;
                 win = load_window(it, w0);
+                ok = publish(it);
             }
             while (L < total && ok) {
                 const int L_next = ws_snake(k + 1, bid, grid);
@@ -399,22 +436,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                     w0_next = nx.key_lo >> p.log2_page;
                     win_next = load_window(nx, w0_next);
                 }
-                // the item's queries: n_rows rows x G heads of kv-head g
-                const uint32_t qs = qc % C::kNQ;
-                if (qc >= (uint32_t)C::kNQ && !mbar_wait(smem_u32(&qempty_bar[qs]), ((qc / C::kNQ) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
-                    s_item[qs] = it;  // published with the queries (the arrive below releases it)
-                    const uint32_t qdst = sbase + C::kOffQ + qs * C::kQBytes;
-                    const uint32_t qbytes = (uint32_t)(p.group * D * 2);
-                    mbar_arrive_expect_tx(smem_u32(&qfull_bar[qs]), qbytes * it.n_rows);
-                    for (int i = 0; i < it.n_rows; ++i)
-                        bulk_load(qdst + i * qbytes, p.q + ((int64_t)(it.q_row + i) * p.hq + it.g * p.group) * D,
-                                  qbytes, smem_u32(&qfull_bar[qs]));
-                }
-                ++qc;
+                bool sent_next = L_next >= total;
                 for (int j0 = it.key_lo; j0 < it.key_hi;) {
                     const int rows = ws_tile_rows<C::TK>(it, j0);
                     const uint32_t st = tc % C::kStages;
@@ -478,7 +500,15 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                     }
                     ++tc;
                     j0 += rows;
+                    if (!sent_next) {
+                        sent_next = true;
+                        if (!publish(nx)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                 }
+                if (ok && !sent_next && !publish(nx)) ok = false;
                 L = L_next;
                 ++k;
                 it = nx;

@@ -104,6 +104,11 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  : "memory");
 }
 
+// Bring the 128-byte line holding `addr` into L2.
+__device__ __forceinline__ void prefetch_l2(const void *addr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(addr) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
