@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     auto sV = [&](int s) { return sbase + C::kOffV + s * C::kKVBytes; };
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     volatile uint32_t *abort_flag = &s_abort;
+    bool sent_row = false;  // this thread sent a staged row with a bulk copy
 
     const int G = p.group, RT = kQM / p.group;  // rows a tile
     // partials: kv-head blockIdx.y; a prompt chunk: the launch order (block
@@ -639,7 +640,22 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
         if (!isfinite(l_sum) || (!PARTIAL && !(l_sum > 0.f))) bad = 1;
         const int64_t u = (int64_t)(q_row + row_i) * p.hq + g * G + (qi % G);
         const int64_t at = u * (PARTIAL ? p.n_splits_max : 1) + split;  // partial slot
+        // O goes out through shared memory when the tile has many rows: each
+        // thread stages its half row in the K/V buffers (free once the last
+        // P V is done; rows padded by 16 bytes, so a warp's 16-byte stores hit
+        // distinct banks) and sends it with one bulk copy, where direct stores
+        // would have each warp instruction touch 32 rows.  A tile of few rows
+        // (under 64 queries) stores directly: its fixed cost is lower.
         const int d0 = h * (D / 2);
+        const bool out16 = !PARTIAL && p.out_bf16;
+        const bool staged = rows_here * G >= 64;
+        constexpr int kRowW = D + 4;  // 32-bit words a staged row (f32; a bf16 row uses half)
+        const uint32_t row_w = out16 ? (uint32_t)(D / 2 + 4) : (uint32_t)kRowW;
+        uint32_t *stage = reinterpret_cast<uint32_t *>(sbase_ptr + C::kOffK) + qi * row_w + (out16 ? d0 / 2 : d0);
+        uint32_t *gout = PARTIAL ? reinterpret_cast<uint32_t *>(p.part_o + at * D + d0)
+                                 : (out16 ? reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d0)
+                                          : reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(p.out) + u * D + d0));
+        const bool direct = !staged && valid_row && !aborted;
         uint32_t obad = 0;
 #pragma unroll 1
         for (int cc = 0; cc < D / 64; ++cc) {
@@ -652,26 +668,19 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
                 o[w] = PARTIAL ? __uint_as_float(r[w]) : __uint_as_float(r[w]) / l_sum;
                 obad |= !isfinite(o[w]);
             }
-            if (valid_row && !aborted) {
-                if (PARTIAL) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.part_o + at * D + d0 + cc * 32);
-#pragma unroll
-                    for (int w = 0; w < 8; ++w)
-                        dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
-                } else if (p.out_bf16) {
-                    uint4 *dst =
-                        reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d0 + cc * 32);
+            if (staged || direct) {
+                uint32_t *dst = staged ? stage : gout;
+                if (out16) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc * 16);
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        dst[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]),
-                                            pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
-                                            pack_bf16x2(o[8 * w + 4], o[8 * w + 5]),
-                                            pack_bf16x2(o[8 * w + 6], o[8 * w + 7]));
+                        d4[w] = make_uint4(pack_bf16x2(o[8 * w], o[8 * w + 1]), pack_bf16x2(o[8 * w + 2], o[8 * w + 3]),
+                                           pack_bf16x2(o[8 * w + 4], o[8 * w + 5]),
+                                           pack_bf16x2(o[8 * w + 6], o[8 * w + 7]));
                 } else {
-                    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d0 + cc * 32);
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + cc * 32);
 #pragma unroll
-                    for (int w = 0; w < 8; ++w)
-                        dst[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
+                    for (int w = 0; w < 8; ++w) d4[w] = make_float4(o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
                 }
             }
         }
@@ -679,6 +688,22 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
         s_xbad[1][h][qi] = obad;
         named_bar_sync(pair_bar, 64);
         bad |= s_xbad[1][0][qi] | s_xbad[1][1][qi];
+        // a flagged prompt row goes out as canonical NaN (partials keep o:
+        // the flag marks them); a CTA that gave up writes it directly, since
+        // copies may still be landing in its buffers
+        if (!PARTIAL && bad && valid_row) {
+            const uint32_t nanw = out16 ? 0x7fc07fc0u : 0x7fc00000u;
+            uint32_t *dst = (staged && !aborted) ? stage : gout;
+            const int words = out16 ? D / 4 : D / 2;
+            for (int w = 0; w < words; w += 4)
+                *reinterpret_cast<uint4 *>(dst + w) = make_uint4(nanw, nanw, nanw, nanw);
+        }
+        if (staged && valid_row && !aborted) {
+            fence_proxy_async_smem();
+            bulk_store(gout, smem_u32(stage), out16 ? (uint32_t)(D / 2) * 2u : (uint32_t)(D / 2) * 4u);
+            bulk_commit();
+            sent_row = true;
+        }
         if (valid_row) {
             if (PARTIAL) {
                 // natural-log reference max, sum, flag: the merge weighs partial
@@ -689,22 +714,11 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
                     p.part_flag[at] = (uint8_t)(bad ? 1 : 0);
                 }
             } else {
-                if (bad) {
-                    const float qnan = __int_as_float(0x7fc00000);
-                    for (int d = d0; d < d0 + D / 2; d += 8) {
-                        if (p.out_bf16)
-                            *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(p.out) + u * D + d) =
-                                make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
-                        else {
-                            float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + u * D + d);
-                            dst[0] = make_float4(qnan, qnan, qnan, qnan);
-                            dst[1] = make_float4(qnan, qnan, qnan, qnan);
-                        }
-                    }
-                }
                 if (p.out_flags && h == 0) p.out_flags[u] = (uint8_t)(bad ? 1 : 0);
             }
         }
+        // (a bulk copy is waited for at the very end, after the tensor
+        // memory is released, so a CTA waiting for its SM starts sooner)
     }
     // everyone: report a timeout, give in-flight work a bounded chance to land,
     // release tensor memory
@@ -724,6 +738,9 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
+    // a thread that sent a staged row stays until the copy has read it from
+    // shared memory; the grid's completion makes its writes visible
+    if (sent_row) bulk_wait_read();
 }
 
 // ---------------------------------------------------------------------------

@@ -109,6 +109,16 @@ __device__ __forceinline__ void prefetch_l2(const void *addr) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(addr) : "memory");
 }
 
+// Bulk copy shared -> global (both 16-byte aligned, bytes a multiple of 16),
+// tracked by the issuing thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every bulk group this thread committed has read its source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
