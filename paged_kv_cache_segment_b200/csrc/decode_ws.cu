@@ -521,312 +521,331 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             }
         }
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-        return;
-    }
-
-    // ---- consumer warps
-    const int gq = lane >> 2, t4 = lane & 3;
-    const float scale_log2 = p.scale_log2;
-    uint32_t tc = 0, qc = 0;
-    for (int k = 0, L = ws_snake(0, bid, grid); L < total; L = ws_snake(++k, bid, grid)) {
-        // the item (resolved by the producer) and its queries -> B fragments
-        // (Q^T), kept in registers
-        const uint32_t qs = qc % C::kNQ;
-        // (no barrier here: a warp that finishes an item's combine late joins
-        // the next item late; a wait that gives up skips the item's tiles and
-        // the loop-end barrier takes every warp out)
-        const bool q_ok = mbar_wait(smem_u32(&qfull_bar[qs]), (qc / C::kNQ) & 1);
-        WsItem it = s_item[qs];
-        if (!q_ok) it.key_lo = it.key_hi = 0;
-        const int q_item = it.n_rows * p.group;
-        uint32_t qb[D / 16][2];
-        {
-            const uint32_t qsrc = sbase + C::kOffQ + qs * C::kQBytes;
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ks += 2) {
-                const uint32_t a = qsrc + (lane & 7) * (D * 2) + (2 * ks + (lane >> 3)) * 16;
-                ldsm_x4(a, qb[ks][0], qb[ks][1], qb[ks + 1][0], qb[ks + 1][1]);
+    } else {
+        // ---- consumer warps
+        const int gq = lane >> 2, t4 = lane & 3;
+        const float scale_log2 = p.scale_log2;
+        uint32_t tc = 0, qc = 0;
+        for (int k = 0, L = ws_snake(0, bid, grid); L < total; L = ws_snake(++k, bid, grid)) {
+            // the item (resolved by the producer) and its queries -> B fragments
+            // (Q^T), kept in registers
+            const uint32_t qs = qc % C::kNQ;
+            // (no barrier here: a warp that finishes an item's combine late joins
+            // the next item late; a wait that gives up skips the item's tiles and
+            // the loop-end barrier takes every warp out)
+            const bool q_ok = mbar_wait(smem_u32(&qfull_bar[qs]), (qc / C::kNQ) & 1);
+            WsItem it = s_item[qs];
+            if (!q_ok) it.key_lo = it.key_hi = 0;
+            const int q_item = it.n_rows * p.group;
+            uint32_t qb[D / 16][2];
+            {
+                const uint32_t qsrc = sbase + C::kOffQ + qs * C::kQBytes;
+    #pragma unroll
+                for (int ks = 0; ks < D / 16; ks += 2) {
+                    const uint32_t a = qsrc + (lane & 7) * (D * 2) + (2 * ks + (lane >> 3)) * 16;
+                    ldsm_x4(a, qb[ks][0], qb[ks][1], qb[ks + 1][0], qb[ks + 1][1]);
+                }
             }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&qempty_bar[qs]));
-        ++qc;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&qempty_bar[qs]));
+            ++qc;
 
-        // per-thread state: queries 2*t4 and 2*t4+1; O^T rows d = 16*mt + gq (+8)
-        const int qa = 2 * t4, qb_ = qa + 1;
-        const int lim_a = qa < q_item ? min(it.key_hi, it.causal0 + qa / p.group) : it.key_hi;
-        const int lim_b = qb_ < q_item ? min(it.key_hi, it.causal0 + qb_ / p.group) : it.key_hi;
-        float o[D / 16][4];
-#pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-        uint32_t e0 = 0, e1 = 0, tb0 = 0, tb1 = 0, badp = 0;
-        const int kb = warp * 16;
-        bool aborted = !q_ok;
+            // per-thread state: queries 2*t4 and 2*t4+1; O^T rows d = 16*mt + gq (+8)
+            const int qa = 2 * t4, qb_ = qa + 1;
+            const int lim_a = qa < q_item ? min(it.key_hi, it.causal0 + qa / p.group) : it.key_hi;
+            const int lim_b = qb_ < q_item ? min(it.key_hi, it.causal0 + qb_ / p.group) : it.key_hi;
+            float o[D / 16][4];
+    #pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+            uint32_t e0 = 0, e1 = 0, tb0 = 0, tb1 = 0, badp = 0;
+            const int kb = warp * 16;
+            bool aborted = !q_ok;
 
-        for (int j0 = it.key_lo; j0 < it.key_hi;) {
-            const int rows = ws_tile_rows<C::TK>(it, j0);
-            const uint32_t st = tc % C::kStages;
-            if (!mbar_wait(smem_u32(&full_bar[st]), (tc / C::kStages) & 1)) {
-                aborted = true;
-                break;
-            }
-            badp |= s_meta[st];
-            const uint32_t sK = sbase + st * C::kStageBytes, sV = sK + C::kTileBytes;
-            bool wrote = false;
-            if (kb < rows) {
-                // clean this warp's V rows: past the tile's keys -> 0; seen by only
-                // some rows and nonfinite -> 0 and flag the rows that see it
-                if (kb + 16 > rows || j0 + kb + 16 > it.full_hi) {
-                    unsigned char *vrows = base_ptr + st * C::kStageBytes + C::kTileBytes;
-                    // rows past the tile's keys hold other keys' values: zero them
-                    for (int idx = lane; idx < 16 * C::kSlabs * 8; idx += 32) {
-                        const int r = kb + idx / (C::kSlabs * 8);
-                        const int rest = idx % (C::kSlabs * 8), sl = rest / 8, ch = rest % 8;
-                        if (r >= rows) {
-                            *reinterpret_cast<uint4 *>(vrows + sl * C::kSlab + r * 128 + ch * 16) =
-                                make_uint4(0, 0, 0, 0);
-                            wrote = true;
-                        }
-                    }
-                    // rows only some of the item's rows see: one lane scans one row;
-                    // a nonfinite row is zeroed and flags the queries that see it
-                    uint32_t nf = 0;
-                    if (lane < 16) {
-                        const int r = kb + lane;
-                        if (r < rows && j0 + r >= it.full_hi) {
-                            for (int sl = 0; sl < C::kSlabs; ++sl) {
-                                const uint4 *rp = reinterpret_cast<const uint4 *>(vrows + sl * C::kSlab + r * 128);
-#pragma unroll
-                                for (int ch = 0; ch < 8; ++ch) {
-                                    const uint4 v = rp[ch];
-                                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e)
-                                        nf |= (((w4[e] & 0x7f80u) == 0x7f80u) ||
-                                               ((w4[e] & 0x7f800000u) == 0x7f800000u))
-                                                  ? 1u
-                                                  : 0u;
-                                }
-                            }
-                            if (nf) {
-                                for (int sl = 0; sl < C::kSlabs; ++sl) {
-                                    uint4 *wp = reinterpret_cast<uint4 *>(vrows + sl * C::kSlab + r * 128);
-#pragma unroll
-                                    for (int ch = 0; ch < 8; ++ch) wp[ch] = make_uint4(0, 0, 0, 0);
-                                }
+            for (int j0 = it.key_lo; j0 < it.key_hi;) {
+                const int rows = ws_tile_rows<C::TK>(it, j0);
+                const uint32_t st = tc % C::kStages;
+                if (!mbar_wait(smem_u32(&full_bar[st]), (tc / C::kStages) & 1)) {
+                    aborted = true;
+                    break;
+                }
+                badp |= s_meta[st];
+                const uint32_t sK = sbase + st * C::kStageBytes, sV = sK + C::kTileBytes;
+                bool wrote = false;
+                if (kb < rows) {
+                    // clean this warp's V rows: past the tile's keys -> 0; seen by only
+                    // some rows and nonfinite -> 0 and flag the rows that see it
+                    if (kb + 16 > rows || j0 + kb + 16 > it.full_hi) {
+                        unsigned char *vrows = base_ptr + st * C::kStageBytes + C::kTileBytes;
+                        // rows past the tile's keys hold other keys' values: zero them
+                        for (int idx = lane; idx < 16 * C::kSlabs * 8; idx += 32) {
+                            const int r = kb + idx / (C::kSlabs * 8);
+                            const int rest = idx % (C::kSlabs * 8), sl = rest / 8, ch = rest % 8;
+                            if (r >= rows) {
+                                *reinterpret_cast<uint4 *>(vrows + sl * C::kSlab + r * 128 + ch * 16) =
+                                    make_uint4(0, 0, 0, 0);
                                 wrote = true;
                             }
                         }
-                    }
-                    const uint32_t badrows = __ballot_sync(0xffffffffu, nf != 0) & 0xffffu;
-                    for (int r = 0; r < 16; ++r)
-                        if ((badrows >> r) & 1u) {
-                            const int key = j0 + kb + r;
-                            if (key < lim_a) tb0 = 1;
-                            if (key < lim_b) tb1 = 1;
+                        // rows only some of the item's rows see: one lane scans one row;
+                        // a nonfinite row is zeroed and flags the queries that see it
+                        uint32_t nf = 0;
+                        if (lane < 16) {
+                            const int r = kb + lane;
+                            if (r < rows && j0 + r >= it.full_hi) {
+                                for (int sl = 0; sl < C::kSlabs; ++sl) {
+                                    const uint4 *rp = reinterpret_cast<const uint4 *>(vrows + sl * C::kSlab + r * 128);
+    #pragma unroll
+                                    for (int ch = 0; ch < 8; ++ch) {
+                                        const uint4 v = rp[ch];
+                                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+                                        for (int e = 0; e < 4; ++e)
+                                            nf |= (((w4[e] & 0x7f80u) == 0x7f80u) ||
+                                                   ((w4[e] & 0x7f800000u) == 0x7f800000u))
+                                                      ? 1u
+                                                      : 0u;
+                                    }
+                                }
+                                if (nf) {
+                                    for (int sl = 0; sl < C::kSlabs; ++sl) {
+                                        uint4 *wp = reinterpret_cast<uint4 *>(vrows + sl * C::kSlab + r * 128);
+    #pragma unroll
+                                        for (int ch = 0; ch < 8; ++ch) wp[ch] = make_uint4(0, 0, 0, 0);
+                                    }
+                                    wrote = true;
+                                }
+                            }
                         }
-                    __syncwarp();
-                }
+                        const uint32_t badrows = __ballot_sync(0xffffffffu, nf != 0) & 0xffffu;
+                        for (int r = 0; r < 16; ++r)
+                            if ((badrows >> r) & 1u) {
+                                const int key = j0 + kb + r;
+                                if (key < lim_a) tb0 = 1;
+                                if (key < lim_b) tb1 = 1;
+                            }
+                        __syncwarp();
+                    }
 
-                // ---- S^T = K Q^T for this warp's 16 keys
-                // two accumulators (even / odd k-steps) halve the MMA dependency chain
-                float s4[4] = {0.f, 0.f, 0.f, 0.f}, s5[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const int r = kb + (lane & 7) + (((lane >> 3) & 1) << 3);
-                    const int ch = 2 * ks + (lane >> 4);
-                    const uint32_t a = sK + (ch >> 3) * C::kSlab + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(a, a0, a1, a2, a3);
-                    if (ks & 1)
-                        mma_bf16(s5, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                    else
-                        mma_bf16(s4, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                }
-                s4[0] += s5[0];
-                s4[1] += s5[1];
-                s4[2] += s5[2];
-                s4[3] += s5[3];
-                // mask, check, online softmax (queries qa, qb_ ; keys rows kb+gq, kb+gq+8)
-                const int ra = kb + gq, rb = ra + 8;
-                const int ka = j0 + ra, kbk = j0 + rb;
-                const bool va0 = ra < rows && ka < lim_a, va1 = ra < rows && ka < lim_b;
-                const bool vb0 = rb < rows && kbk < lim_a, vb1 = rb < rows && kbk < lim_b;
-                float x0 = s4[0] * scale_log2, x1 = s4[1] * scale_log2, x2 = s4[2] * scale_log2,
-                      x3 = s4[3] * scale_log2;
-                e0 = max(e0, max(va0 ? exp_bits(x0) : 0u, vb0 ? exp_bits(x2) : 0u));
-                e1 = max(e1, max(va1 ? exp_bits(x1) : 0u, vb1 ? exp_bits(x3) : 0u));
-                x0 = va0 ? x0 : -INFINITY;
-                x1 = va1 ? x1 : -INFINITY;
-                x2 = vb0 ? x2 : -INFINITY;
-                x3 = vb1 ? x3 : -INFINITY;
-                float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-                for (int o_ = 4; o_ < 32; o_ <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
-                }
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-                const float al0 = ex2(m0 - mu0), al1 = ex2(m1 - mu1);
-                m0 = mn0;
-                m1 = mn1;
-                const float p0 = ex2(x0 - mu0), p1 = ex2(x1 - mu1), p2 = ex2(x2 - mu0), p3 = ex2(x3 - mu1);
-                l0 = l0 * al0 + p0 + p2;
-                l1 = l1 * al1 + p1 + p3;
-                if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
+                    // ---- S^T = K Q^T for this warp's 16 keys
+                    // two accumulators (even / odd k-steps) halve the MMA dependency chain
+                    float s4[4] = {0.f, 0.f, 0.f, 0.f}, s5[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const int r = kb + (lane & 7) + (((lane >> 3) & 1) << 3);
+                        const int ch = 2 * ks + (lane >> 4);
+                        const uint32_t a = sK + (ch >> 3) * C::kSlab + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(a, a0, a1, a2, a3);
+                        if (ks & 1)
+                            mma_bf16(s5, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                        else
+                            mma_bf16(s4, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                    }
+                    s4[0] += s5[0];
+                    s4[1] += s5[1];
+                    s4[2] += s5[2];
+                    s4[3] += s5[3];
+                    // mask, check, online softmax (queries qa, qb_ ; keys rows kb+gq, kb+gq+8)
+                    const int ra = kb + gq, rb = ra + 8;
+                    const int ka = j0 + ra, kbk = j0 + rb;
+                    const bool va0 = ra < rows && ka < lim_a, va1 = ra < rows && ka < lim_b;
+                    const bool vb0 = rb < rows && kbk < lim_a, vb1 = rb < rows && kbk < lim_b;
+                    float x0 = s4[0] * scale_log2, x1 = s4[1] * scale_log2, x2 = s4[2] * scale_log2,
+                          x3 = s4[3] * scale_log2;
+                    e0 = max(e0, max(va0 ? exp_bits(x0) : 0u, vb0 ? exp_bits(x2) : 0u));
+                    e1 = max(e1, max(va1 ? exp_bits(x1) : 0u, vb1 ? exp_bits(x3) : 0u));
+                    x0 = va0 ? x0 : -INFINITY;
+                    x1 = va1 ? x1 : -INFINITY;
+                    x2 = vb0 ? x2 : -INFINITY;
+                    x3 = vb1 ? x3 : -INFINITY;
+                    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+    #pragma unroll
+                    for (int o_ = 4; o_ < 32; o_ <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
+                    }
+                    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                    const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0, mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
+                    const float al0 = ex2(m0 - mu0), al1 = ex2(m1 - mu1);
+                    m0 = mn0;
+                    m1 = mn1;
+                    const float p0 = ex2(x0 - mu0), p1 = ex2(x1 - mu1), p2 = ex2(x2 - mu0), p3 = ex2(x3 - mu1);
+                    l0 = l0 * al0 + p0 + p2;
+                    l1 = l1 * al1 + p1 + p3;
+                    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+    #pragma unroll
+                        for (int mt = 0; mt < D / 16; ++mt) {
+                            o[mt][0] *= al0;
+                            o[mt][1] *= al1;
+                            o[mt][2] *= al0;
+                            o[mt][3] *= al1;
+                        }
+                    }
+                    // P^T fragments: (keys 2t4.., query gq) from (key gq.., queries 2t4..)
+                    const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+                    const uint32_t r01 = pack_bf16x2(p0 - bf16_lo_to_f32(h01), p1 - bf16_hi_to_f32(h01));
+                    const uint32_t r23 = pack_bf16x2(p2 - bf16_lo_to_f32(h23), p3 - bf16_hi_to_f32(h23));
+                    const uint32_t bh0 = movmatrix_t(h01), bh1 = movmatrix_t(h23);
+                    const uint32_t bl0 = movmatrix_t(r01), bl1 = movmatrix_t(r23);
+                    // ---- O^T += V^T P^T
+    #pragma unroll
                     for (int mt = 0; mt < D / 16; ++mt) {
-                        o[mt][0] *= al0;
-                        o[mt][1] *= al1;
-                        o[mt][2] *= al0;
-                        o[mt][3] *= al1;
+                        const int r = kb + (lane & 7) + ((lane >> 4) << 3);
+                        const int ch = 2 * mt + ((lane >> 3) & 1);
+                        const uint32_t a = sV + (ch >> 3) * C::kSlab + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_t(a, a0, a1, a2, a3);
+                        mma_bf16(o[mt], a0, a1, a2, a3, bh0, bh1);
+                        mma_bf16(o[mt], a0, a1, a2, a3, bl0, bl1);
                     }
                 }
-                // P^T fragments: (keys 2t4.., query gq) from (key gq.., queries 2t4..)
-                const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-                const uint32_t r01 = pack_bf16x2(p0 - bf16_lo_to_f32(h01), p1 - bf16_hi_to_f32(h01));
-                const uint32_t r23 = pack_bf16x2(p2 - bf16_lo_to_f32(h23), p3 - bf16_hi_to_f32(h23));
-                const uint32_t bh0 = movmatrix_t(h01), bh1 = movmatrix_t(h23);
-                const uint32_t bl0 = movmatrix_t(r01), bl1 = movmatrix_t(r23);
-                // ---- O^T += V^T P^T
-#pragma unroll
-                for (int mt = 0; mt < D / 16; ++mt) {
-                    const int r = kb + (lane & 7) + ((lane >> 4) << 3);
-                    const int ch = 2 * mt + ((lane >> 3) & 1);
-                    const uint32_t a = sV + (ch >> 3) * C::kSlab + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(a, a0, a1, a2, a3);
-                    mma_bf16(o[mt], a0, a1, a2, a3, bh0, bh1);
-                    mma_bf16(o[mt], a0, a1, a2, a3, bl0, bl1);
-                }
+                __syncwarp();
+                if (wrote) fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
+                ++tc;
+                j0 += rows;
             }
-            __syncwarp();
-            if (wrote) fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
-            ++tc;
-            j0 += rows;
-        }
-        if (named_bar_red_or(1, C::NC * 32, aborted)) {  // every consumer warp leaves together
-            if (tid == 0) atomicOr(p.status, TF_DEV_TIMEOUT);
-            break;
-        }
+            if (named_bar_red_or(1, C::NC * 32, aborted)) {  // every consumer warp leaves together
+                if (tid == 0) {
+                    atomicOr(p.status, TF_DEV_TIMEOUT);
+                    s_abort = 1;
+                }
+                break;
+            }
 
-        // ---- combine the four warps (tree through shared memory) and write
-#pragma unroll
-        for (int o_ = 4; o_ < 32; o_ <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, o_);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, o_);
-            e0 = max(e0, __shfl_xor_sync(0xffffffffu, e0, o_));
-            e1 = max(e1, __shfl_xor_sync(0xffffffffu, e1, o_));
-            tb0 |= __shfl_xor_sync(0xffffffffu, tb0, o_);
-            tb1 |= __shfl_xor_sync(0xffffffffu, tb1, o_);
-        }
-        uint32_t f0 = (e0 == 0x7f800000u) | tb0 | badp, f1 = (e1 == 0x7f800000u) | tb1 | badp;
-        auto put = [&](int slot) {
-            float *dst = comb_o + slot * kWsQ * C::kCombStride;
-#pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                dst[qa * C::kCombStride + 16 * mt + gq] = o[mt][0];
-                dst[qb_ * C::kCombStride + 16 * mt + gq] = o[mt][1];
-                dst[qa * C::kCombStride + 16 * mt + gq + 8] = o[mt][2];
-                dst[qb_ * C::kCombStride + 16 * mt + gq + 8] = o[mt][3];
-            }
-            if (gq == 0) {
-                comb_m[slot][qa] = m0;
-                comb_m[slot][qb_] = m1;
-                comb_l[slot][qa] = l0;
-                comb_l[slot][qb_] = l1;
-                comb_f[slot][qa] = f0;
-                comb_f[slot][qb_] = f1;
-            }
-        };
-        auto take = [&](int slot) {
-            const float *src = comb_o + slot * kWsQ * C::kCombStride;
-            const float ma = comb_m[slot][qa], mb = comb_m[slot][qb_];
-            const float la = comb_l[slot][qa], lb = comb_l[slot][qb_];
-            f0 |= comb_f[slot][qa];
-            f1 |= comb_f[slot][qb_];
-            const float M0 = fmaxf(m0, ma), M1 = fmaxf(m1, mb);
-            const float u0 = (M0 == -INFINITY) ? 0.f : M0, u1 = (M1 == -INFINITY) ? 0.f : M1;
-            const float w0 = ex2(m0 - u0), w1 = ex2(m1 - u1), wa = ex2(ma - u0), wb = ex2(mb - u1);
-            l0 = l0 * w0 + la * wa;
-            l1 = l1 * w1 + lb * wb;
-            m0 = M0;
-            m1 = M1;
-#pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                o[mt][0] = o[mt][0] * w0 + src[qa * C::kCombStride + 16 * mt + gq] * wa;
-                o[mt][1] = o[mt][1] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq] * wb;
-                o[mt][2] = o[mt][2] * w0 + src[qa * C::kCombStride + 16 * mt + gq + 8] * wa;
-                o[mt][3] = o[mt][3] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq + 8] * wb;
-            }
-        };
-        // Warps 2 and 3 hand their states to warps 0 and 1 and go on to the
-        // next item; warp 1 then hands its state to warp 0, which writes the
-        // item's partials from its registers.  The slots are free again before
-        // the next item's combine: every warp passes the loop-end barrier first.
-        if (warp >= 2) put(warp - 2);
-        named_bar_sync(1, C::NC * 32);
-        if (warp < 2) {
-            take(warp);
-            named_bar_sync(2, 64);  // warp 0 has read slot 0: warp 1 may refill it
-            if (warp == 1) put(0);
-            named_bar_sync(2, 64);
-        }
-        if (warp == 0) {
-            take(0);
-            bool nf0 = !isfinite(l0), nf1 = !isfinite(l1);
-#pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                nf0 |= !isfinite(o[mt][0]) || !isfinite(o[mt][2]);
-                nf1 |= !isfinite(o[mt][1]) || !isfinite(o[mt][3]);
-            }
-#pragma unroll
+            // ---- combine the four warps (tree through shared memory) and write
+    #pragma unroll
             for (int o_ = 4; o_ < 32; o_ <<= 1) {
-                nf0 |= __shfl_xor_sync(0xffffffffu, nf0, o_);
-                nf1 |= __shfl_xor_sync(0xffffffffu, nf1, o_);
+                l0 += __shfl_xor_sync(0xffffffffu, l0, o_);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, o_);
+                e0 = max(e0, __shfl_xor_sync(0xffffffffu, e0, o_));
+                e1 = max(e1, __shfl_xor_sync(0xffffffffu, e1, o_));
+                tb0 |= __shfl_xor_sync(0xffffffffu, tb0, o_);
+                tb1 |= __shfl_xor_sync(0xffffffffu, tb1, o_);
             }
-            f0 |= nf0;
-            f1 |= nf1;
-            // this lane's queries qa, qb_ and dims 16 mt + gq (+ 8): eight
-            // consecutive floats of a row per four lanes
-            auto slot_of = [&](int qq) {
-                const int i = qq / p.group, hl = qq - i * p.group;
-                const int64_t u = RING ? (int64_t)it.s * p.hq + it.g * p.group + hl
-                                       : (int64_t)(it.q_row + i) * p.hq + it.g * p.group + hl;
-                return u * p.n_splits_max + it.c;
+            uint32_t f0 = (e0 == 0x7f800000u) | tb0 | badp, f1 = (e1 == 0x7f800000u) | tb1 | badp;
+            auto put = [&](int slot) {
+                float *dst = comb_o + slot * kWsQ * C::kCombStride;
+    #pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    dst[qa * C::kCombStride + 16 * mt + gq] = o[mt][0];
+                    dst[qb_ * C::kCombStride + 16 * mt + gq] = o[mt][1];
+                    dst[qa * C::kCombStride + 16 * mt + gq + 8] = o[mt][2];
+                    dst[qb_ * C::kCombStride + 16 * mt + gq + 8] = o[mt][3];
+                }
+                if (gq == 0) {
+                    comb_m[slot][qa] = m0;
+                    comb_m[slot][qb_] = m1;
+                    comb_l[slot][qa] = l0;
+                    comb_l[slot][qb_] = l1;
+                    comb_f[slot][qa] = f0;
+                    comb_f[slot][qb_] = f1;
+                }
             };
-            if (qa < q_item) {
-                const int64_t at = slot_of(qa);
-                float *dst = p.part_o + at * D;
-#pragma unroll
+            auto take = [&](int slot) {
+                const float *src = comb_o + slot * kWsQ * C::kCombStride;
+                const float ma = comb_m[slot][qa], mb = comb_m[slot][qb_];
+                const float la = comb_l[slot][qa], lb = comb_l[slot][qb_];
+                f0 |= comb_f[slot][qa];
+                f1 |= comb_f[slot][qb_];
+                const float M0 = fmaxf(m0, ma), M1 = fmaxf(m1, mb);
+                const float u0 = (M0 == -INFINITY) ? 0.f : M0, u1 = (M1 == -INFINITY) ? 0.f : M1;
+                const float w0 = ex2(m0 - u0), w1 = ex2(m1 - u1), wa = ex2(ma - u0), wb = ex2(mb - u1);
+                l0 = l0 * w0 + la * wa;
+                l1 = l1 * w1 + lb * wb;
+                m0 = M0;
+                m1 = M1;
+    #pragma unroll
                 for (int mt = 0; mt < D / 16; ++mt) {
-                    dst[16 * mt + gq] = o[mt][0];
-                    dst[16 * mt + gq + 8] = o[mt][2];
+                    o[mt][0] = o[mt][0] * w0 + src[qa * C::kCombStride + 16 * mt + gq] * wa;
+                    o[mt][1] = o[mt][1] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq] * wb;
+                    o[mt][2] = o[mt][2] * w0 + src[qa * C::kCombStride + 16 * mt + gq + 8] * wa;
+                    o[mt][3] = o[mt][3] * w1 + src[qb_ * C::kCombStride + 16 * mt + gq + 8] * wb;
                 }
-                if (gq == 0) {
-                    p.part_m[at] = (m0 == -INFINITY) ? -INFINITY : m0 * kLn2;
-                    p.part_l[at] = l0;
-                    p.part_flag[at] = (uint8_t)(f0 ? 1 : 0);
+            };
+            // Warps 2 and 3 hand their states to warps 0 and 1 and go on to the
+            // next item; warp 1 then hands its state to warp 0, which writes the
+            // item's partials from its registers.  The slots are free again before
+            // the next item's combine: every warp passes the loop-end barrier first.
+            if (warp >= 2) put(warp - 2);
+            named_bar_sync(1, C::NC * 32);
+            if (warp < 2) {
+                take(warp);
+                named_bar_sync(2, 64);  // warp 0 has read slot 0: warp 1 may refill it
+                if (warp == 1) put(0);
+                named_bar_sync(2, 64);
+            }
+            if (warp == 0) {
+                take(0);
+                bool nf0 = !isfinite(l0), nf1 = !isfinite(l1);
+    #pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    nf0 |= !isfinite(o[mt][0]) || !isfinite(o[mt][2]);
+                    nf1 |= !isfinite(o[mt][1]) || !isfinite(o[mt][3]);
+                }
+    #pragma unroll
+                for (int o_ = 4; o_ < 32; o_ <<= 1) {
+                    nf0 |= __shfl_xor_sync(0xffffffffu, nf0, o_);
+                    nf1 |= __shfl_xor_sync(0xffffffffu, nf1, o_);
+                }
+                f0 |= nf0;
+                f1 |= nf1;
+                // this lane's queries qa, qb_ and dims 16 mt + gq (+ 8): eight
+                // consecutive floats of a row per four lanes
+                auto slot_of = [&](int qq) {
+                    const int i = qq / p.group, hl = qq - i * p.group;
+                    const int64_t u = RING ? (int64_t)it.s * p.hq + it.g * p.group + hl
+                                           : (int64_t)(it.q_row + i) * p.hq + it.g * p.group + hl;
+                    return u * p.n_splits_max + it.c;
+                };
+                if (qa < q_item) {
+                    const int64_t at = slot_of(qa);
+                    float *dst = p.part_o + at * D;
+    #pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        dst[16 * mt + gq] = o[mt][0];
+                        dst[16 * mt + gq + 8] = o[mt][2];
+                    }
+                    if (gq == 0) {
+                        p.part_m[at] = (m0 == -INFINITY) ? -INFINITY : m0 * kLn2;
+                        p.part_l[at] = l0;
+                        p.part_flag[at] = (uint8_t)(f0 ? 1 : 0);
+                    }
+                }
+                if (qb_ < q_item) {
+                    const int64_t at = slot_of(qb_);
+                    float *dst = p.part_o + at * D;
+    #pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) {
+                        dst[16 * mt + gq] = o[mt][1];
+                        dst[16 * mt + gq + 8] = o[mt][3];
+                    }
+                    if (gq == 0) {
+                        p.part_m[at] = (m1 == -INFINITY) ? -INFINITY : m1 * kLn2;
+                        p.part_l[at] = l1;
+                        p.part_flag[at] = (uint8_t)(f1 ? 1 : 0);
+                    }
                 }
             }
-            if (qb_ < q_item) {
-                const int64_t at = slot_of(qb_);
-                float *dst = p.part_o + at * D;
-#pragma unroll
-                for (int mt = 0; mt < D / 16; ++mt) {
-                    dst[16 * mt + gq] = o[mt][1];
-                    dst[16 * mt + gq + 8] = o[mt][3];
-                }
-                if (gq == 0) {
-                    p.part_m[at] = (m1 == -INFINITY) ? -INFINITY : m1 * kLn2;
-                    p.part_l[at] = l1;
-                    p.part_flag[at] = (uint8_t)(f1 ? 1 : 0);
-                }
-            }
+        }
+    }
+
+    // ---- a CTA that gave up (a bounded wait ran out) must not leave while
+    // copies it issued are still landing in its shared memory: each stage's
+    // and query buffer's barrier gets a bounded wait for the phase it is in
+    // (a TMA box or bulk copy in flight completes it; an idle one times out
+    // after 20 ms), then the CTA exits
+    __syncthreads();
+    if (s_abort && tid == 0) {
+        for (int i = 0; i < C::kStages; ++i) {
+            mbar_wait(smem_u32(&full_bar[i]), 0u, 20000000ull);
+            mbar_wait(smem_u32(&full_bar[i]), 1u, 20000000ull);
+        }
+        for (int i = 0; i < C::kNQ; ++i) {
+            mbar_wait(smem_u32(&qfull_bar[i]), 0u, 20000000ull);
+            mbar_wait(smem_u32(&qfull_bar[i]), 1u, 20000000ull);
         }
     }
 }
