@@ -701,7 +701,7 @@ def bench_ring(wl, tf, dev, steps, peaks, traffic, cpu_s):
     cpu = oracle_cpu(lambda: orc.ring_attn(b.q, b.ring_k, b.ring_v, b.rsegs, b.scale), cpu_s, kv / 1e9, "GB/s",
                      "whole passes of the 17 rings")
     return {"workload": "drafter ring: 17 rows, rings of 4,200 slots, random heads, U{1000..4200} valid, 16/2 heads, "
-                        "D256, 256-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
+                        "D256, 384-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
             "ms_per_step": round(ms, 5), "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
             "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                  traffic.get("decode_ws:drafter_ring")), "cpu_baseline": cpu,
@@ -801,12 +801,13 @@ def bench_prompt(wl, tf, dev, steps, peaks, traffic, cpu_s):
 def bench_block(wl, tf, dev, steps, peaks, traffic, cpu_s):
     """A drafter-block round: 16 streams, each a block of 9 rows seeing all of
     its stream's keys (the FULL rule), contexts U{1,024..8,192}, 32/8 heads,
-    D 128, pages of 32, 512-key partials + merge; 3 rotating copies."""
+    D 128, pages of 32, 768-key partials (the fastest of 512-2,048 in a sweep
+    on a B200) + merge; 3 rotating copies."""
     import oracle
 
     b0 = wl.multi_stream_decode(2)
     keys = [int(x) for x in b0.segs[:, 2]]
-    b = wl.make_paged_batch(12, [9] * len(keys), keys, 32, 8, 128, 32, unused="nan", split_keys=512)
+    b = wl.make_paged_batch(12, [9] * len(keys), keys, 32, 8, 128, 32, unused="nan", split_keys=768)
     run = DecodeRun(b, dev)
 
     def step(k):
@@ -830,7 +831,7 @@ def bench_block(wl, tf, dev, steps, peaks, traffic, cpu_s):
                                             sel=sel), cpu_s, kv / b.n_kv_heads / 1e9, "GB/s",
                      "kv-head 0 of every block (all rows, its 4 q-heads)")
     return {"workload": "drafter blocks: 16 streams x 9 rows, every row over all its stream's keys, contexts "
-                        "U{1024..8192}, 32/8 heads, D128, P32, 512-key partials + merge",
+                        "U{1024..8192}, 32/8 heads, D128, P32, 768-key partials + merge",
             "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2), "ms_per_step": round(ms, 5),
             "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                       traffic.get("prompt_tc:drafter_block")),
