@@ -428,15 +428,21 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                 ok = publish(it);
             }
             while (L < total && ok) {
+                // the next item is resolved, its page ids requested and its
+                // queries published once this item's first tile has gone out
+                // (so a CTA's first copy waits on nothing but its own page ids)
                 const int L_next = ws_snake(k + 1, bid, grid);
                 WsItem nx{};
                 int win_next = 0, w0_next = 0;
-                if (L_next < total) {  // requested now, used when the next item starts
+                bool sent_next = false;
+                auto prep_next = [&]() -> bool {
+                    sent_next = true;
+                    if (L_next >= total) return true;
                     nx = ws_resolve<RING>(p, prefix, prefix_full, tail_order, n_full, L_next);
                     w0_next = nx.key_lo >> p.log2_page;
                     win_next = load_window(nx, w0_next);
-                }
-                bool sent_next = L_next >= total;
+                    return publish(nx);
+                };
                 for (int j0 = it.key_lo; j0 < it.key_hi;) {
                     const int rows = ws_tile_rows<C::TK>(it, j0);
                     const uint32_t st = tc % C::kStages;
@@ -500,15 +506,12 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                     }
                     ++tc;
                     j0 += rows;
-                    if (!sent_next) {
-                        sent_next = true;
-                        if (!publish(nx)) {
-                            ok = false;
-                            break;
-                        }
+                    if (!sent_next && !prep_next()) {
+                        ok = false;
+                        break;
                     }
                 }
-                if (ok && !sent_next && !publish(nx)) ok = false;
+                if (ok && !sent_next && !prep_next()) ok = false;
                 L = L_next;
                 ++k;
                 it = nx;
