@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--only", default="", help="comma list: decode,verify,ring,tree,prompt,argmax,block,append,e2e,cpu")
-    ap.add_argument("--secondary-steps", type=int, default=20)
+    ap.add_argument("--secondary-steps", type=int, default=24)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--secondary-cpu-seconds", type=float, default=3.0,
                     help="seconds of oracle time beside each secondary workload (0: one repetition)")
@@ -259,20 +259,6 @@ def timed_steps(launches, steps):
     return per, total
 
 
-def b2b_ms(fn, steps):
-    """Average milliseconds of fn(k) over `steps` calls issued back to back,
-    with CUDA events at the two ends only (no event between launches)."""
-    import torch
-
-    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for k in range(steps):
-        fn(k)
-    z.record()
-    torch.cuda.synchronize()
-    return a.elapsed_time(z) / steps
-
-
 def graph_replayer(fn, copies):
     """Capture fn(k) for each input copy k in a CUDA graph (after one eager
     warm-up call each, which also loads the kernels) and return
@@ -299,6 +285,39 @@ def graph_replayer(fn, copies):
 
     replay.graphs = graphs
     return replay
+
+
+def chain_replayer(fn, copies):
+    """Capture fn(0), ..., fn(copies - 1) back to back in ONE CUDA graph
+    (after an eager call of each, which also loads the kernels): consecutive
+    steps then meet at a kernel boundary inside a graph, as in a serving loop
+    that captures its decode steps, rather than at a graph launch, which costs
+    the device a few microseconds of idle time per launch.  Returns
+    run(steps) -> device milliseconds of exactly `steps` steps: steps // copies
+    replays of the chain, then the remaining steps one graph each (step k
+    always reads input copy k % copies), with CUDA events at the two ends."""
+    import torch
+
+    single = graph_replayer(fn, copies)
+    chain = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(chain, capture_error_mode="thread_local"):
+        for k in range(copies):
+            fn(k)
+
+    def run(steps):
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps // copies):
+            chain.replay()
+        for k in range(steps - steps % copies, steps):
+            single(k)
+        z.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(z)
+
+    run.single = single
+    run.chain = chain
+    return run
 
 
 def time_cpu(fn, seconds, min_reps=1):
@@ -344,28 +363,35 @@ def bench_headline(args, wl, dev, world, peaks, traffic, barrier, max_over_ranks
     b = wl.multi_stream_decode(2)
     kv_bytes = b.kv_bytes()
     run = DecodeRun(b, dev)
-    # the step (partials + merge), and each kernel alone, captured once per
-    # input copy and replayed: the timed loop has no host work between steps
-    step_g = graph_replayer(run.step, len(run.sets))
-    part_g = graph_replayer(run.partial, len(run.sets))
-    merge_g = graph_replayer(run.merge, len(run.sets))
+    # the step (partials + merge) captured three steps to a graph (one per
+    # input copy) and replayed: the timed loop has no host work between steps,
+    # and steps meet at kernel boundaries inside a graph; each kernel alone,
+    # and the step as one graph launch each, for the record
+    n_sets = len(run.sets)
+    step_c = chain_replayer(run.step, n_sets)
+    part_c = chain_replayer(run.partial, n_sets)
+    step_g = step_c.single
+    part_g = part_c.single
+    merge_g = graph_replayer(run.merge, n_sets)
     for k in range(max(3, args.warmup)):
         step_g(k)
+    step_c(n_sets)
     barrier()
     sampler = ClockSampler(local)
     result = None
     for attempt in range(2):
         sampler.start()
         barrier()
-        # the step, timed at its ends only (an event between the two launches
-        # would stop the merge from overlapping the partial kernel's tail)
-        _, total = timed_steps([step_g], args.steps)
+        # the timed region: exactly K steps, events at its two ends
+        total = step_c(args.steps)
         barrier()
-        # each kernel alone: events around every launch, and the partial
-        # kernel's launches back to back (events at the ends only), whose
-        # average duration is the roofline's denominator
+        # the partial kernel's launches back to back (chained the same way),
+        # whose average duration is the roofline's denominator; then each
+        # kernel with events around every launch, and the step as its own
+        # graph launch
+        part_b2b = part_c(args.steps) / args.steps
         per, _ = timed_steps([part_g, merge_g], args.steps)
-        part_b2b = b2b_ms(part_g, args.steps)
+        _, total_each = timed_steps([step_g], args.steps)
         barrier()
         clocks = sampler.stop()
         if not clocks_bad(clocks) or attempt == 1:
@@ -378,6 +404,7 @@ def bench_headline(args, wl, dev, world, peaks, traffic, barrier, max_over_ranks
     eager_ms = max_over_ranks(eager_total) / n_eager
     total_max = max_over_ranks(total)
     part_ms = part_b2b
+    each_ms = max_over_ranks(total_each) / args.steps
     ms_step = total_max / args.steps
     assert int(run.st.item()) == 0, "device status set during the decode bench"
     value = whole_job_gbs(kv_bytes, world, ms_step)
@@ -394,9 +421,12 @@ def bench_headline(args, wl, dev, world, peaks, traffic, barrier, max_over_ranks
                     "decode_partial_ms_events_each": round(per[0] / args.steps, 5),
                     "merge_ms_alone": round(per[1] / args.steps, 5),
                     "merge_ms_in_step": round(ms_step - part_ms, 5),
-                    "timing": "decode_partial_ms: the partial kernel's launches back to back, events at the ends; "
-                              "*_events_each / merge_ms_alone: events around every launch"},
-        "launch": "each step replays a CUDA graph of the two kernels, one graph per input copy",
+                    "timing": "decode_partial_ms: the partial kernel's launches back to back (chained graphs), "
+                              "events at the ends; *_events_each / merge_ms_alone: events around every launch"},
+        "launch": "CUDA graphs of three consecutive steps (one per input copy, two kernels a step) replayed back "
+                  "to back; K steps = K // 3 replays + the rest one step-graph each",
+        "graph_each_step": {"ms_per_step": round(each_ms, 5), "value": round(whole_job_gbs(kv_bytes, world, each_ms), 2),
+                            "path": "every step its own graph launch, an event between steps"},
         "eager": {"value": round(whole_job_gbs(kv_bytes, world, eager_ms), 2), "ms_per_step": round(eager_ms, 5),
                   "steps": n_eager, "path": "the same two calls issued through the Python binding every step"},
         "peaks_source": peaks["source"],
@@ -608,12 +638,18 @@ def bench_verify(wl, dev, steps, peaks, traffic, cpu_s):
     logits = wl.verify_logits(3, rows)
     run = DecodeRun(b, dev, logits, copies=8)  # 8 x (151 MB of KV + 17 MB of logits)
     n = len(run.sets)
-    part_g, merge_g, arg_g = (graph_replayer(f, n) for f in (run.partial, run.merge, run.argmax))
+    part_c, arg_c = chain_replayer(run.partial, n), chain_replayer(run.argmax, n)
+    pm_c = chain_replayer(lambda k: (run.partial(k), run.merge(k)), n)
+    three_c = chain_replayer(lambda k: (run.partial(k), run.merge(k), run.argmax(k)), n)
+    part_g, arg_g = part_c.single, arg_c.single
+    merge_g = graph_replayer(run.merge, n)
     for k in range(3):
         part_g(k)
         merge_g(k)
         arg_g(k)
-    per, total = timed_steps([part_g, merge_g, arg_g], steps)
+    per, _ = timed_steps([part_g, merge_g, arg_g], steps)
+    pm_ms = pm_c(steps) / steps  # the verify step: partials + merge
+    three_ms = three_c(steps) / steps  # the round as three calls
 
     # the same round as one call (tf_verify_round): merge and argmax launch as
     # programmatic dependents, timed at the round's ends
@@ -624,13 +660,13 @@ def bench_verify(wl, dev, steps, peaks, traffic, cpu_s):
                            part_flag=run.pf, out=run.out, flags=run.fl, status=run.st, logits=x["logits"],
                            ids=run.ids, id_flags=run.afl, segs_host=b.segs)
 
-    round_g = graph_replayer(round_call, n)
-    round_g(0)
-    _, round_total = timed_steps([round_g], steps)
-    # each kernel's launches back to back over the 8 copies, events at the
-    # ends only: the average launch duration, the rooflines' denominator
-    part_b2b = b2b_ms(part_g, steps)
-    arg_b2b = b2b_ms(arg_g, steps)
+    round_c = chain_replayer(round_call, n)
+    round_ms = round_c(steps) / steps
+    # each kernel's launches back to back over the 8 copies (chained graphs),
+    # events at the ends only: the average launch duration, the rooflines'
+    # denominator
+    part_b2b = part_c(steps) / steps
+    arg_b2b = arg_c(steps) / steps
     kv = b.kv_bytes()
     pms, mms, ams = per[0] / steps, per[1] / steps, per[2] / steps
     flops = 4 * b.head_dim * sum(int(s[1]) * b.n_q_heads * (int(s[2]) - int(s[1]) + 1) + b.n_q_heads *
@@ -645,7 +681,8 @@ def bench_verify(wl, dev, steps, peaks, traffic, cpu_s):
         "verify": {"workload": "shared verify: 8 streams x U{1..16} rows, 16/2 heads, D256, P32, contexts "
                                f"U{{2048..16384}}, {split}-key partials (tf_choose_split_keys) + merge", "rows": rows,
                    "split_keys": split,
-                   "kv_gbs": round(kv / (pms + mms) / 1e6, 2), "ms_per_step": round((pms + mms), 5),
+                   "kv_gbs": round(kv / pm_ms / 1e6, 2), "ms_per_step": round(pm_ms, 5),
+                   "ms_per_step_events_each": round(pms + mms, 5),
                    "tflops": round(flops / (part_b2b * 1e-3) / 1e12, 2),
                    "partial_ms": round(part_b2b, 5), "partial_ms_events_each": round(pms, 5),
                    "roofline": dict(roofline("hbm", kv / (part_b2b * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
@@ -654,8 +691,8 @@ def bench_verify(wl, dev, steps, peaks, traffic, cpu_s):
                    "cpu_baseline": cpu_verify,
                    "launches": 2 * steps, "l2": "8 rotating copies"},
         "round": {"workload": "the shared verify round in one call: partials, merge, argmax of its 62 rows",
-                  "ms": round(round_total / steps, 5), "ms_three_calls": round(total / steps, 5),
-                  "kv_plus_logit_gbs": round((kv + arg_bytes) / (round_total / steps) / 1e6, 2),
+                  "ms": round(round_ms, 5), "ms_three_calls": round(three_ms, 5),
+                  "kv_plus_logit_gbs": round((kv + arg_bytes) / round_ms / 1e6, 2),
                   "launches": 3 * steps},
         "argmax": {"workload": f"{rows} rows x 128,000 bf16 ~N(0,3), ties in ~1/4 of rows",
                    "rows_per_s": round(rows / (arg_b2b * 1e-3), 1), "ms": round(arg_b2b, 5),
@@ -690,11 +727,10 @@ def bench_ring(wl, tf, dev, steps, peaks, traffic, cpu_s):
         tf.tf_ring_attn(x["q"], x["rk"], x["rv"], x["rs"], scale=b.scale, split_slots=b.split_slots,
                         n_splits_max=b.n_splits_max, workspace=ws, out=out, flags=fl, status=st, rsegs_host=b.rsegs)
 
-    g = graph_replayer(step, 3)
-    for k in range(3):
-        g(k)
-    per, total = timed_steps([g], steps)
-    ms = total / steps
+    c = chain_replayer(step, 3)
+    c(3)
+    ms = c(steps) / steps
+    _, total_each = timed_steps([c.single], steps)
     kv = b.kv_bytes()
     assert int(st.item()) == 0
     orc = oracle.get()
@@ -702,7 +738,8 @@ def bench_ring(wl, tf, dev, steps, peaks, traffic, cpu_s):
                      "whole passes of the 17 rings")
     return {"workload": "drafter ring: 17 rows, rings of 4,200 slots, random heads, U{1000..4200} valid, 16/2 heads, "
                         "D256, 384-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
-            "ms_per_step": round(ms, 5), "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
+            "ms_per_step": round(ms, 5), "ms_per_step_graph_each": round(total_each / steps, 5),
+            "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
             "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                  traffic.get("decode_ws:drafter_ring")), "cpu_baseline": cpu,
             "launches": 2 * steps, "l2": "3 rotating copies"}
@@ -732,11 +769,10 @@ def bench_tree(wl, tf, dev, steps, peaks, traffic, cpu_s):
                              n_splits_max=b.n_splits_max, workspace=ws, out=out, flags=fl, status=st,
                              tsegs_host=b.tsegs, parents_host=b.parents)
 
-    g = graph_replayer(step, 3)
-    for k in range(3):
-        g(k)
-    _, total = timed_steps([g], steps)
-    ms = total / steps
+    c = chain_replayer(step, 3)
+    c(3)
+    ms = c(steps) / steps
+    _, total_each = timed_steps([c.single], steps)
     kv = b.kv_bytes()
     assert int(st.item()) == 0
     orc = oracle.get()
@@ -746,6 +782,7 @@ def bench_tree(wl, tf, dev, steps, peaks, traffic, cpu_s):
                         "U{1000..4184} slots of 4,200-slot rings, 16/2 heads, D256, "
                         f"{b.split_slots}-slot partials + merge", "nodes": rows,
             "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2), "ms_per_step": round(ms, 5),
+            "ms_per_step_graph_each": round(total_each / steps, 5),
             "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                       traffic.get("prompt_tc:drafter_trees")),
                              kernel="prompt_tc_kernel<256, hilo, partial, tree> + merge (the whole step)"),
@@ -772,10 +809,10 @@ def bench_prompt(wl, tf, dev, steps, peaks, traffic, cpu_s):
             tf.tf_paged_attn_prompt(x["q"], x["kp"], x["vp"], x["pt"], sg, scale=b.scale, out=out, flags=fl,
                                     status=st)
 
-    g = graph_replayer(step, 2)
-    g(0)
-    per, total = timed_steps([g], steps)
-    ms = total / steps
+    c = chain_replayer(step, 2)
+    c(2)
+    ms = c(steps) / steps
+    _, total_each = timed_steps([c.single], steps)
     n = rows
     flops = 4 * d * hq * n * (n + 1) // 2
     assert int(st.item()) == 0
@@ -789,6 +826,7 @@ def bench_prompt(wl, tf, dev, steps, peaks, traffic, cpu_s):
                      sample_flops / 1e12, "TFLOP/s", "the prompt's last 32 rows x 16 heads (14,969-15,000 keys each)")
     return {"workload": "long causal prompt: 15,000 tokens in 2,048-row chunks, 16/4 heads, D256, P32, 469 shuffled "
                         "pages, bf16 out", "tflops": round(tfl, 2), "ms_per_step": round(ms, 4),
+            "ms_per_step_graph_each": round(total_each / steps, 4),
             "algorithmic_flops": flops,
             "roofline": dict(roofline("tensor", tfl, peaks["bf16_tflops"], "TFLOP/s",
                                       traffic.get("prompt_tc:long_prompt")), kernel="prompt_tc_kernel<256, bf16>",
@@ -817,11 +855,10 @@ def bench_block(wl, tf, dev, steps, peaks, traffic, cpu_s):
                                part_l=run.pl, part_flag=run.pf, status=run.st, segs_host=b.segs)
         run.merge(k)
 
-    g = graph_replayer(step, len(run.sets))
-    for k in range(3):
-        g(k)
-    _, total = timed_steps([g], steps)
-    ms = total / steps
+    c = chain_replayer(step, len(run.sets))
+    c(len(run.sets))
+    ms = c(steps) / steps
+    _, total_each = timed_steps([c.single], steps)
     kv = b.kv_bytes()
     assert int(run.st.item()) == 0
     orc = oracle.get()
@@ -833,6 +870,7 @@ def bench_block(wl, tf, dev, steps, peaks, traffic, cpu_s):
     return {"workload": "drafter blocks: 16 streams x 9 rows, every row over all its stream's keys, contexts "
                         "U{1024..8192}, 32/8 heads, D128, P32, 768-key partials + merge",
             "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2), "ms_per_step": round(ms, 5),
+            "ms_per_step_graph_each": round(total_each / steps, 5),
             "roofline": dict(roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",
                                       traffic.get("prompt_tc:drafter_block")),
                              kernel="prompt_tc_kernel<128, hilo, partial> + merge (the whole step)"),
@@ -868,11 +906,10 @@ def bench_append(wl, tf, dev, steps, peaks, traffic, cpu_s):
         kp, vp = pools[k % 3]
         tf.tf_kv_append(kr, vr, kp, vp, pt, sd, status=st, segs_host=sh)
 
-    g = graph_replayer(step, 3)
-    for k in range(3):
-        g(k)
-    _, total = timed_steps([g], steps)
-    ms = total / steps
+    c = chain_replayer(step, 3)
+    c(3)
+    ms = c(steps) / steps
+    _, total_each = timed_steps([c.single], steps)
     moved = 2 * 2 * n * hkv * d * 2  # K and V, read from the rows and written into the pages
     assert int(st.item()) == 0
     gbs = moved / (ms * 1e-3) / 1e9
@@ -881,6 +918,7 @@ def bench_append(wl, tf, dev, steps, peaks, traffic, cpu_s):
                      "GB/s", "whole appends of the 15,000 rows (the oracle copies both pools first)")
     return {"workload": "append the 15,000-token prompt's K/V rows into 469 shuffled pages of 32 in one call "
                         "(4 kv-heads, D256)", "gbs": round(gbs, 2), "ms_per_step": round(ms, 5),
+            "ms_per_step_graph_each": round(total_each / steps, 5),
             "bytes_per_step": moved, "roofline": dict(roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s",
                                                                traffic.get("kv_append:long_prompt")),
                                                       kernel="kv_append_kernel<256>"),
