@@ -12,14 +12,15 @@
 // on the 32-bit words it holds in registers, two bf16 values each:
 // max.bf16x2 keeps the largest value of each half and max.u16x2 over the
 // magnitude bits the largest exponent pattern (reaching 0x7f80 means a NaN or
-// an infinity); the thread's largest value M_t is then looked for again among
-// its own words with an IEEE compare (so -0 equals +0), which gives the
-// first column holding it.  A thread's candidate is the pair (key(M_t),
-// column), where key is an order-preserving 16-bit image of the value with
-// -0 mapped to +0's key: the row's answer is the largest key and, among equal
-// keys, the smallest column.  Warps and then the CTA reduce the pairs; each
-// CTA stores its pair into rank 0's shared memory (distributed shared
-// memory), one cluster barrier, and rank 0 writes the id and the flag.
+// an infinity).  Values compare through key, an order-preserving 16-bit
+// image with -0 mapped to +0's key.  The CTA's largest key comes from the
+// warps' maxima (one barrier); then only the threads whose own largest value
+// it is look for it again among their words with an IEEE compare (so -0
+// equals +0), and the smallest column any of them finds is the CTA's first
+// column holding it (a warp with none of those threads skips the search).
+// The row's answer is the largest key and, among equal keys, the smallest
+// column: each CTA stores its pair into rank 0's shared memory (distributed
+// shared memory), one cluster barrier, and rank 0 writes the id and flag.
 //
 // A first split cluster barrier (arrive at entry, wait before the first
 // remote store) makes sure every CTA of the cluster has started before any of
@@ -91,7 +92,7 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __shared__ uint32_t w_key[kArgWarps], w_bad[kArgWarps];
-    __shared__ int w_col[kArgWarps];
+    __shared__ int s_col;  // the CTA's first column holding its largest value
     // rank 0's slots, filled by every CTA of the cluster, two buffers by row parity
     __shared__ uint32_t x_key[2][kArgmaxCluster], x_bad[2][kArgmaxCluster];
     __shared__ int x_col[2][kArgmaxCluster];
@@ -150,10 +151,26 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
         }
         // nonfinite: some half's magnitude pattern reached the all-ones exponent
         const uint32_t bad = ((mag & 0xffffu) >= 0x7f80u || (mag >> 16) >= 0x7f80u) ? 1u : 0u;
-        uint32_t key = max(key16(vmax & 0xffffu), key16(vmax >> 16));
-        // ---- the first of the thread's columns holding its largest value
-        const uint32_t M = unkey16(key), M2 = M | (M << 16);
+        const uint32_t key = max(key16(vmax & 0xffffu), key16(vmax >> 16));
+        // ---- the CTA's largest key: warps, then every warp over the warps'
+        const uint32_t wbad = __reduce_or_sync(0xffffffffu, bad);
+        {
+            const uint32_t wkey = __reduce_max_sync(0xffffffffu, key);
+            if (lane == 0) {
+                w_key[warp] = wkey;
+                w_bad[warp] = wbad;
+            }
+        }
+        if (it == 0 && tid == 0) s_col = INT_MAX;
+        __syncthreads();
+        const uint32_t ckey = __reduce_max_sync(0xffffffffu, w_key[lane]);  // kArgWarps == 32: a lane a warp
+        // ---- the first column holding the CTA's largest value, looked for
+        // again only by the threads whose own largest value it is (a warp with
+        // none of them skips the search)
+        if (__any_sync(0xffffffffu, key == ckey)) {
         int col = INT_MAX;
+        if (key == ckey) {
+        const uint32_t M = unkey16(ckey), M2 = M | (M << 16);
         if constexpr (VEC) {
 #pragma unroll
             for (int j = 0; j < kArgBatch * 4; ++j) {
@@ -173,14 +190,11 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
         }
         for (int c = (VEC ? (v1 << 3) : c0) + tid; c < c1 && col == INT_MAX; c += kArgThreads)
             if (eq_bf16x2(rp[c], M) & 0xffffu) col = c;
-        // ---- the CTA's pair, then the cluster's on rank 0
-        warp_best(key, col);
-        const uint32_t wbad = __reduce_or_sync(0xffffffffu, bad);
-        if (lane == 0) {
-            w_key[warp] = key;
-            w_col[warp] = col;
-            w_bad[warp] = wbad;
         }
+        col = __reduce_min_sync(0xffffffffu, col);
+        if (lane == 0) atomicMin(&s_col, col);
+        }
+        // ---- the CTA's pair, then the cluster's on rank 0
         if (!joined) {
             asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
             joined = true;
@@ -188,14 +202,12 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
         __syncthreads();
         const int buf = it & 1;
         if (warp == 0) {
-            uint32_t k = w_key[lane];  // kArgWarps == 32: a lane a warp
-            int c = w_col[lane];
             const uint32_t b = __reduce_or_sync(0xffffffffu, w_bad[lane]);
-            warp_best(k, c);
             if (lane == 0) {
-                *cluster.map_shared_rank(&x_key[buf][rank], 0) = k;
-                *cluster.map_shared_rank(&x_col[buf][rank], 0) = c;
+                *cluster.map_shared_rank(&x_key[buf][rank], 0) = ckey;
+                *cluster.map_shared_rank(&x_col[buf][rank], 0) = s_col;
                 *cluster.map_shared_rank(&x_bad[buf][rank], 0) = b;
+                s_col = INT_MAX;  // for the next row (read here, set again after its first barrier)
             }
         }
         cluster.sync();

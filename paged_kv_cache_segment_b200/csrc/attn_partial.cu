@@ -568,10 +568,12 @@ __global__ void __launch_bounds__(kThreads, (D == 256) ? 1 : 2) attn_partial_ker
 // Lane c holds partial c's weight e^(m_c - M) (0 for an empty partial); the o
 // rows are then read with independent, predicated loads four partials at a
 // time.  The kernel may be launched as a programmatic dependent of the
-// partial kernel: it waits for that grid before reading.
+// partial kernel: it waits for that grid before it reads a partial or writes
+// anything.  A ring or tree merge reads its table entry before that wait:
+// the partial kernel before it never writes the table, and that kernel
+// started only after all earlier work on the stream had finished.
 template <int D, int MODE>
 __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     // a dependent launch (a verify round's argmax) may start; it waits for
     // this grid's completion before it reads anything
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -588,6 +590,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
     int64_t out_u = u, pu = u;  // the output row's unit, the partials' unit
     int C = p.n_parts;
     const float qnan = __int_as_float(0x7fc00000);
+    if constexpr (MODE == kMergeRows) asm volatile("griddepcontrol.wait;" ::: "memory");
     if constexpr (MODE == kMergeRing) {
         // only rows the table names are written; a bad entry (the partial
         // kernel skipped it) gives a flagged NaN row
@@ -598,6 +601,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
         const bool bad = e.size <= 0 || e.n_valid < 1 || e.n_valid > e.size || e.head < 0 || e.head >= e.size ||
                          e.base < 0 || e.base + e.size > p.ring_slots_total ||
                          (e.n_valid + p.split_slots - 1) / p.split_slots > p.n_parts;
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         if (bad) {
             for (int d0 = dbase + lane * 4; d0 < dbase + DW; d0 += 128)
                 *reinterpret_cast<float4 *>(p.out + out_u * D + d0) = make_float4(qnan, qnan, qnan, qnan);
@@ -617,6 +621,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
         out_u = pu = (int64_t)(e.q_row + i) * p.hq + h;
         const bool ok = tree_seg_ok(e, p.n_rows_total, p.n_parents, p.ring_slots_total) &&
                         tree_splits(e, p.split_slots).n_sp <= p.n_parts;
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         if (!ok) {
             for (int d0 = dbase + lane * 4; d0 < dbase + DW; d0 += 128)
                 *reinterpret_cast<float4 *>(p.out + out_u * D + d0) = make_float4(qnan, qnan, qnan, qnan);
