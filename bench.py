@@ -737,7 +737,7 @@ def bench_ring(wl, tf, dev, steps, peaks, traffic, cpu_s):
     cpu = oracle_cpu(lambda: orc.ring_attn(b.q, b.ring_k, b.ring_v, b.rsegs, b.scale), cpu_s, kv / 1e9, "GB/s",
                      "whole passes of the 17 rings")
     return {"workload": "drafter ring: 17 rows, rings of 4,200 slots, random heads, U{1000..4200} valid, 16/2 heads, "
-                        "D256, 384-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
+                        "D256, 320-slot partials + merge", "kv_gbs": round(kv / (ms * 1e-3) / 1e9, 2),
             "ms_per_step": round(ms, 5), "ms_per_step_graph_each": round(total_each / steps, 5),
             "pages_ms_reference": "0.24 ms a 4,200-slot draft step on GB10 (one stream)",
             "roofline": roofline("hbm", kv / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s",

@@ -545,7 +545,7 @@ def drafter_trees(seed: int = 6, n_streams: int = 17, unused: str = "nan", split
     )
 
 
-def drafter_ring(seed: int = 5, n_streams: int = 17, unused: str = "nan", split_slots: int = 384) -> RingBatch:
+def drafter_ring(seed: int = 5, n_streams: int = 17, unused: str = "nan", split_slots: int = 320) -> RingBatch:
     """17 one-row streams, each over its own ring of 4,200 slots with a random
     write head; valid counts U{1,000..4,200}; 16/2 heads, D 256."""
     return make_ring_batch(
