@@ -9,12 +9,15 @@ is one decode pass over that batch: the split-KV partial kernel and the merge.
 value = KV bytes a step reads (every visible key once per kv-head) / step time,
 in GB/s, with inputs resident in HBM; three copies of the batch rotate between
 steps (906 MB of KV, over seven times the L2), so no step finds its data in L2.
-Each timed step replays a CUDA graph holding the step's kernels (one graph per
-input copy, captured from the public calls), so the Python binding's host work
-never sits between two steps on the device; the same calls issued eagerly are
-reported beside it.  A kernel's roofline divides its algorithmic bytes (or
-FLOPs) by its average duration over launches issued back to back, CUDA events
-at the two ends.  At N > 1 every rank runs its own replica of the batch
+The timed steps replay CUDA graphs captured from the public calls, three
+consecutive steps to a graph (one per input copy), so the Python binding's
+host work never sits between two steps on the device and consecutive steps
+meet at a kernel boundary inside a graph, as in a serving loop that captures
+its steps; K steps are K // 3 graph replays plus the rest one step-graph
+each.  The same step as one graph launch a step, and the calls issued
+eagerly, are reported beside it.  A kernel's roofline divides its
+algorithmic bytes (or FLOPs) by its average duration over launches issued
+back to back, CUDA events at the two ends.  At N > 1 every rank runs its own replica of the batch
 (independent streams, no collective on the data path) and value = all ranks'
 bytes / the slowest rank's time ("weak" scaling).
 
