@@ -456,6 +456,19 @@ TF_API const char *tf_status_str(tf_status s);
 /* ABI version of this header: bumped when a signature changes. */
 TF_API int32_t tf_abi_version(void);
 
+/*
+ * Test hook for the bounded waits, so failure detection can be tested
+ * without a fault: while on != 0, the warp-specialized and tensor-core
+ * kernels launched from the calling host thread (decode, block and verify
+ * partials, ring, tree and prompt calls) issue none of their loads, so the
+ * waits of their other warps run out after 5 ms.  Each such launch reports
+ * TF_DEV_TIMEOUT in its status word, leaves the outputs it did not reach
+ * unwritten or flagged (a prompt chunk's rows come out as flagged NaN), and
+ * leaves the device usable: no copy or MMA is in flight when its CTAs exit.
+ * on = 0 restores normal launches.  Needed only by tests; TF_OK always.
+ */
+TF_API tf_status tf_wait_limit_test(int32_t on);
+
 #ifdef __cplusplus
 }
 #endif

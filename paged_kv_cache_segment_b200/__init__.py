@@ -26,4 +26,5 @@ from .binding import (  # noqa: F401
     tf_choose_split_keys,
     tf_status_str,
     tf_verify_round,
+    tf_wait_limit_test,
 )

@@ -21,13 +21,13 @@ LIB_PATH = os.path.join(HERE, "libtfpaged.so")
 TF_OK = 0
 STATUS_NAMES = {0: "TF_OK", 1: "TF_ERR_ARG", 2: "TF_ERR_PAST_PAGES", 3: "TF_ERR_BAD_PAGE", 4: "TF_ERR_UNSUPPORTED",
                 5: "TF_ERR_CUDA", 6: "TF_ERR_ALIGN", 7: "TF_ERR_WORKSPACE"}
-TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS = 1, 2, 4, 8
+TF_DEV_BAD_SEG, TF_DEV_PAST_PAGES, TF_DEV_BAD_PAGE, TF_DEV_SPLITS, TF_DEV_TIMEOUT = 1, 2, 4, 8, 16
 TF_OUT_F32, TF_OUT_BF16 = 0, 1
 
 EXPORTS = ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge",
            "tf_paged_attn_prompt", "tf_ring_attn", "tf_ring_workspace_bytes", "tf_ring_tree_attn",
            "tf_ring_tree_workspace_bytes", "tf_ring_attn_noalloc", "tf_argmax_rows", "tf_choose_split_keys",
-           "tf_status_str", "tf_abi_version")
+           "tf_status_str", "tf_abi_version", "tf_wait_limit_test")
 # bytes of the scratch array tf_ring_attn_noalloc keeps in the library's device image
 TF_RING_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -80,6 +80,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.tf_status_str.argtypes = [ctypes.c_int]
     lib.tf_status_str.restype = ctypes.c_char_p
     lib.tf_abi_version.restype = ctypes.c_int32
+    lib.tf_wait_limit_test.argtypes = [ctypes.c_int32]
+    lib.tf_wait_limit_test.restype = ctypes.c_int
     for name in ("tf_paged_attn_decode", "tf_paged_attn_block", "tf_kv_append", "tf_verify_round", "tf_attn_merge", "tf_paged_attn_prompt", "tf_ring_attn",
                  "tf_ring_attn_noalloc", "tf_ring_tree_attn", "tf_argmax_rows", "tf_choose_split_keys"):
         getattr(lib, name).restype = ctypes.c_int
@@ -369,3 +371,9 @@ def tf_status_str(code: int) -> str:
 
 def tf_abi_version() -> int:
     return int(load().tf_abi_version())
+
+
+def tf_wait_limit_test(on: bool) -> None:
+    """Test hook: while on, kernels launched from this host thread issue no
+    loads and their bounded waits run out after 5 ms (TF_DEV_TIMEOUT)."""
+    _check("tf_wait_limit_test", load().tf_wait_limit_test(1 if on else 0))

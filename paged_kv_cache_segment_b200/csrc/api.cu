@@ -12,6 +12,15 @@
 
 using namespace tfp;
 
+// The timeout test hook: per host thread, so a test that turns it on touches
+// no other thread's launches.
+namespace tfp {
+namespace {
+thread_local uint64_t g_wait_runout_ns = 0;
+}
+uint64_t test_wait_runout_ns() { return g_wait_runout_ns; }
+}  // namespace tfp
+
 namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -713,5 +722,10 @@ const char *tf_status_str(tf_status s) {
 }
 
 int32_t tf_abi_version(void) { return 1; }
+
+tf_status tf_wait_limit_test(int32_t on) {
+    tfp::g_wait_runout_ns = on ? 5000000ull : 0ull;  // 5 ms
+    return TF_OK;
+}
 
 }  // extern "C"

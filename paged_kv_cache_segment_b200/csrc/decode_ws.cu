@@ -244,6 +244,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
     __shared__ uint32_t s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t lim = p.wait_ns ? p.wait_ns : 2000000000ull;  // every bounded wait's limit
     const uint32_t sraw = smem_u32(smem_raw);
     const uint32_t sbase = (sraw + 1023u) & ~1023u;
     unsigned char *base_ptr = smem_raw + (sbase - sraw);
@@ -385,8 +386,9 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
         // The whole warp walks the items; lane 0 issues the copies.  Page ids
         // come a window of 32 at a time (one coalesced load by the warp), and
         // the next item's window is requested before the current item's tiles
-        // are issued, so no tile waits on a page-table read.
-        {
+        // are issued, so no tile waits on a page-table read.  (Under the
+        // timeout test hook it issues nothing: the consumers' waits run out.)
+        if (!p.test_idle) {
             const int P = 1 << p.log2_page, BR = P < C::TK ? P : C::TK, n_box = C::TK / BR;
             auto load_window = [&](const WsItem &w, int w0) -> int {
                 if constexpr (RING) {
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             // while item k's tiles stream
             auto publish = [&](const WsItem &w) -> bool {
                 const uint32_t qs = qc % C::kNQ;
-                if (qc >= (uint32_t)C::kNQ && !mbar_wait(smem_u32(&qempty_bar[qs]), ((qc / C::kNQ) - 1) & 1))
+                if (qc >= (uint32_t)C::kNQ && !mbar_wait(smem_u32(&qempty_bar[qs]), ((qc / C::kNQ) - 1) & 1, lim))
                     return false;
                 if (lane == 0) {
                     s_item[qs] = w;  // published with the queries (the arrive below releases it)
@@ -447,7 +449,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
                     const int rows = ws_tile_rows<C::TK>(it, j0);
                     const uint32_t st = tc % C::kStages;
                     if (tc >= (uint32_t)C::kStages &&
-                        !mbar_wait(smem_u32(&empty_bar[st]), ((tc / C::kStages) - 1) & 1)) {
+                        !mbar_wait(smem_u32(&empty_bar[st]), ((tc / C::kStages) - 1) & 1, lim)) {
                         ok = false;
                         break;
                     }
@@ -536,7 +538,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             // (no barrier here: a warp that finishes an item's combine late joins
             // the next item late; a wait that gives up skips the item's tiles and
             // the loop-end barrier takes every warp out)
-            const bool q_ok = mbar_wait(smem_u32(&qfull_bar[qs]), (qc / C::kNQ) & 1);
+            const bool q_ok = mbar_wait(smem_u32(&qfull_bar[qs]), (qc / C::kNQ) & 1, lim);
             WsItem it = s_item[qs];
             if (!q_ok) it.key_lo = it.key_hi = 0;
             const int q_item = it.n_rows * p.group;
@@ -568,7 +570,7 @@ __global__ void __launch_bounds__(WsCfg<D>::kThreads, WsCfg<D>::kMinBlocks)
             for (int j0 = it.key_lo; j0 < it.key_hi;) {
                 const int rows = ws_tile_rows<C::TK>(it, j0);
                 const uint32_t st = tc % C::kStages;
-                if (!mbar_wait(smem_u32(&full_bar[st]), (tc / C::kStages) & 1)) {
+                if (!mbar_wait(smem_u32(&full_bar[st]), (tc / C::kStages) & 1, lim)) {
                     aborted = true;
                     break;
                 }
@@ -901,7 +903,12 @@ static cudaError_t launch_ws_t(const WsParams &p, const void *k, const void *v, 
     if (e != cudaSuccess) return e;
     int64_t grid = ws_grid_cap<D, RING>();
     if (n_items_bound < grid) grid = n_items_bound < 1 ? 1 : n_items_bound;
-    kern<<<(unsigned)grid, WsCfg<D>::kThreads, WsCfg<D>::kSmem, st>>>(mk, mv, p);
+    WsParams q = p;
+    if (const uint64_t runout = test_wait_runout_ns()) {
+        q.test_idle = 1;
+        q.wait_ns = runout;
+    }
+    kern<<<(unsigned)grid, WsCfg<D>::kThreads, WsCfg<D>::kSmem, st>>>(mk, mv, q);
     return cudaGetLastError();
 }
 

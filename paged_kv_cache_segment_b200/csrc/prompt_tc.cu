@@ -86,9 +86,9 @@ struct PTCfg {
 
 // Bounded wait that gives up at once after any thread of the CTA gave up, so
 // every role keeps its barrier sequence without waiting twice the timeout.
-__device__ __forceinline__ bool pt_wait(uint32_t bar, uint32_t phase, volatile uint32_t *abort_flag) {
+__device__ __forceinline__ bool pt_wait(uint32_t bar, uint32_t phase, volatile uint32_t *abort_flag, uint64_t lim) {
     if (*abort_flag) return false;
-    if (mbar_wait(bar, phase)) return true;
+    if (mbar_wait(bar, phase, lim)) return true;
     *abort_flag = 1;
     return false;
 }
@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     __shared__ int s_par[TREE ? kTreeMaxNodes : 1];  // a draft tree's parents
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint64_t lim = p.wait_ns ? p.wait_ns : 2000000000ull;  // every bounded wait's limit
     // the merge that follows may launch now; it waits for this grid to finish
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
     };
 
     // every lane of a helper warp waits; the answer is the warp's, so all lanes branch alike
-    auto wwait = [&](uint32_t b, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(b, phase, abort_flag)); };
+    auto wwait = [&](uint32_t b, uint32_t phase) { return __all_sync(0xffffffffu, pt_wait(b, phase, abort_flag, lim)); };
     if (warp == kPTTmaWarp) {
         // ================= TMA warp: the K/V boxes of a tile go out one per lane,
         // so one warp instruction issues all of them; a buffer is refilled as
@@ -329,7 +330,8 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             __syncwarp();
             if (id >= 0) tma_load_4d(dst0 + sl * kKVSlab + x * BR * 128, map, full, 64 * sl, key0 & (P - 1), g, id);
         };
-        for (int t = 0; t < n_tiles; ++t) {
+        // (under the timeout test hook it issues nothing: the other warps' waits run out)
+        for (int t = 0; t < n_tiles && !p.test_idle; ++t) {
             const int s = t % kKVStages;
             const uint32_t fph = (uint32_t)((t / kKVStages - 1) & 1);  // completion of tile t - kKVStages
             // K(t) once QK(t - stages) has read the buffer, V(t) once P V(t - stages) has
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
                 }
                 if (!moved) {
                     const bool give_up = __any_sync(0xffffffffu, *abort_flag != 0 ||
-                                                                   global_ns() - t_poll > 2000000000ull);
+                                                                   global_ns() - t_poll > lim);
                     if (give_up) {
                         *abort_flag = 1;
                         break;
@@ -484,7 +486,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             const uint32_t ph = (uint32_t)((j >> 1) & 1);
             const uint32_t colS = b ? kColS1 : kColS0;
             const int kh = kt + 32 * h;  // this half's first key
-            pt_wait(bar(kBarS + b), ph, abort_flag);
+            pt_wait(bar(kBarS + b), ph, abort_flag, lim);
             tc_fence_after();
             float sv[32];
             {
@@ -563,7 +565,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             // O holds the tiles before this one: rescale it once P V(j-1) is
             // done; this half rescales O columns h * D/2 .. (h + 1) * D/2 - 1
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                pt_wait(bar(kBarO + ((j - 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1), abort_flag);
+                pt_wait(bar(kBarO + ((j - 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1), abort_flag, lim);
                 tc_fence_after();
 #pragma unroll 1
                 for (int c = 0; c < D / 64; ++c) {
@@ -580,7 +582,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
             // V rows this tile must not feed into P V: past every row's keys ->
             // zero; seen by only some rows and nonfinite -> zero and flag
             if (kt + kBN > full_hi) {
-                pt_wait(bar(kBarVFull + j % kKVStages), (uint32_t)((j / kKVStages) & 1), abort_flag);
+                pt_wait(bar(kBarVFull + j % kKVStages), (uint32_t)((j / kKVStages) & 1), abort_flag, lim);
                 named_bar_sync(1, kPTSoftmax);
                 if (tid == 0) s_vbad[0] = s_vbad[1] = 0;
                 named_bar_sync(1, kPTSoftmax);
@@ -628,7 +630,7 @@ __global__ void __launch_bounds__(kPTThreads, pt_paired<D, PARTIAL>() ? 2 : 1)
 
         // ---- epilogue: the halves' sums and findings meet, then each half
         // stores its D/2 columns of O (divided by the sum, or raw for a partial)
-        if (n_tiles > 0) pt_wait(bar(kBarO + ((n_tiles - 1) & 1)), (uint32_t)(((n_tiles - 1) >> 1) & 1), abort_flag);
+        if (n_tiles > 0) pt_wait(bar(kBarO + ((n_tiles - 1) & 1)), (uint32_t)(((n_tiles - 1) >> 1) & 1), abort_flag, lim);
         tc_fence_after();
         const bool aborted = *abort_flag != 0;
         s_xl[h][qi] = l_run;
@@ -775,8 +777,13 @@ static cudaError_t launch_tc_t(const PromptTcParams &p, const void *k, const voi
     }
     const dim3 grid = PARTIAL ? dim3((unsigned)(p.n_qt * p.n_splits_max), (unsigned)p.hkv, (unsigned)n_segs)
                               : dim3((unsigned)((p.n_rows + RT - 1) / RT), (unsigned)p.hkv);
+    PromptTcParams q = p;
+    if (const uint64_t runout = test_wait_runout_ns()) {
+        q.test_idle = 1;
+        q.wait_ns = runout;
+    }
     if (PARTIAL) {
-        kern<<<grid, kPTThreads, C::kSmemBytes, st>>>(mk, mv, p);
+        kern<<<grid, kPTThreads, C::kSmemBytes, st>>>(mk, mv, q);
         return cudaGetLastError();
     }
     // A prompt chunk may start while the call before it on the stream (this
@@ -794,7 +801,7 @@ static cudaError_t launch_tc_t(const PromptTcParams &p, const void *k, const voi
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, kern, mk, mv, q);
 }
 
 cudaError_t launch_prompt_tc(const PromptTcParams &p, int head_dim, const void *k, const void *v, cudaStream_t st) {
@@ -846,7 +853,12 @@ static cudaError_t launch_tree_t(const PromptTcParams &p, const void *k, const v
         if (e != cudaSuccess) return e;
     }
     const dim3 grid((unsigned)(p.n_qt * p.n_splits_max), (unsigned)p.hkv, (unsigned)n_segs);
-    kern<<<grid, kPTThreads, C::kSmemBytes, st>>>(mk, mv, p);
+    PromptTcParams q = p;
+    if (const uint64_t runout = test_wait_runout_ns()) {
+        q.test_idle = 1;
+        q.wait_ns = runout;
+    }
+    kern<<<grid, kPTThreads, C::kSmemBytes, st>>>(mk, mv, q);
     return cudaGetLastError();
 }
 

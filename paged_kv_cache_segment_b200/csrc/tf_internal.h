@@ -76,6 +76,10 @@ struct PromptTcParams {
     const int32_t *parents;
     int n_parents;
     int64_t ring_slots_total;
+    // the timeout test hook (tf_wait_limit_test): the TMA warp issues nothing
+    // and every bounded wait gives up after wait_ns (0: the 2 s default)
+    int test_idle;
+    uint64_t wait_ns;
 };
 
 // Parameters of the KV append (rows into their pages).
@@ -106,6 +110,10 @@ struct WsParams {
     float *part_o, *part_m, *part_l;
     uint8_t *part_flag;
     uint32_t *status;
+    // the timeout test hook (tf_wait_limit_test): the producer issues nothing
+    // and every bounded wait gives up after wait_ns (0: the 2 s default)
+    int test_idle;
+    uint64_t wait_ns;
 };
 
 struct ArgmaxParams {
@@ -115,6 +123,11 @@ struct ArgmaxParams {
     int32_t *ids;
     uint8_t *flags;
 };
+
+// The timeout test hook: while set (tf_wait_limit_test), the warp-specialized
+// and tensor-core kernels launched on this host thread issue no loads and
+// give up their bounded waits after this many nanoseconds (0: hook off).
+uint64_t test_wait_runout_ns();
 
 cudaError_t launch_attn_partial(const AttnParams &p, int head_dim, bool ring, bool direct, dim3 grid,
                                 cudaStream_t st);
