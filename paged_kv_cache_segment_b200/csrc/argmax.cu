@@ -152,7 +152,8 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
         // nonfinite: some half's magnitude pattern reached the all-ones exponent
         const uint32_t bad = ((mag & 0xffffu) >= 0x7f80u || (mag >> 16) >= 0x7f80u) ? 1u : 0u;
         const uint32_t key = max(key16(vmax & 0xffffu), key16(vmax >> 16));
-        // ---- the CTA's largest key: warps, then every warp over the warps'
+        // ---- the CTA's largest key: each warp's maximum, then every warp
+        // reduces the 32 warps' (one barrier)
         const uint32_t wbad = __reduce_or_sync(0xffffffffu, bad);
         {
             const uint32_t wkey = __reduce_max_sync(0xffffffffu, key);
@@ -167,32 +168,33 @@ __global__ void __cluster_dims__(kArgmaxCluster, 1, 1) __launch_bounds__(kArgThr
         // ---- the first column holding the CTA's largest value, looked for
         // again only by the threads whose own largest value it is (a warp with
         // none of them skips the search)
-        if (__any_sync(0xffffffffu, key == ckey)) {
-        int col = INT_MAX;
-        if (key == ckey) {
-        const uint32_t M = unkey16(ckey), M2 = M | (M << 16);
-        if constexpr (VEC) {
+        auto first_col = [&](uint32_t M) -> int {
+            const uint32_t M2 = M | (M << 16);
+            int col = INT_MAX;
+            if constexpr (VEC) {
 #pragma unroll
-            for (int j = 0; j < kArgBatch * 4; ++j) {
-                const uint32_t e = eq_bf16x2(words[j], M2);
-                const int v = v0 + tid + (j >> 2) * kArgThreads;
-                if (col == INT_MAX && e && v < v1) col = v * 8 + (j & 3) * 2 + ((e & 0xffffu) ? 0 : 1);
-            }
-            for (int v = v0 + tid + kArgBatch * kArgThreads; v < v1 && col == INT_MAX; v += kArgThreads) {
-                const uint4 x = __ldg(vp + v);
-                const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+                for (int j = 0; j < kArgBatch * 4; ++j) {
+                    const uint32_t e = eq_bf16x2(words[j], M2);
+                    const int v = v0 + tid + (j >> 2) * kArgThreads;
+                    if (col == INT_MAX && e && v < v1) col = v * 8 + (j & 3) * 2 + ((e & 0xffffu) ? 0 : 1);
+                }
+                for (int v = v0 + tid + kArgBatch * kArgThreads; v < v1 && col == INT_MAX; v += kArgThreads) {
+                    const uint4 x = __ldg(vp + v);
+                    const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t e = eq_bf16x2(wd[q], M2);
-                    if (col == INT_MAX && e) col = v * 8 + 2 * q + ((e & 0xffffu) ? 0 : 1);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t e = eq_bf16x2(wd[q], M2);
+                        if (col == INT_MAX && e) col = v * 8 + 2 * q + ((e & 0xffffu) ? 0 : 1);
+                    }
                 }
             }
-        }
-        for (int c = (VEC ? (v1 << 3) : c0) + tid; c < c1 && col == INT_MAX; c += kArgThreads)
-            if (eq_bf16x2(rp[c], M) & 0xffffu) col = c;
-        }
-        col = __reduce_min_sync(0xffffffffu, col);
-        if (lane == 0) atomicMin(&s_col, col);
+            for (int c = (VEC ? (v1 << 3) : c0) + tid; c < c1 && col == INT_MAX; c += kArgThreads)
+                if (eq_bf16x2(rp[c], M) & 0xffffu) col = c;
+            return col;
+        };
+        if (__any_sync(0xffffffffu, key == ckey)) {
+            const int col = __reduce_min_sync(0xffffffffu, key == ckey ? first_col(unkey16(ckey)) : INT_MAX);
+            if (lane == 0) atomicMin(&s_col, col);
         }
         // ---- the CTA's pair, then the cluster's on rank 0
         if (!joined) {
